@@ -1,0 +1,243 @@
+"""fp64 CPU oracle for the DCP LSE-weighted combine (pack, combine, unpack+combine).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the bench's CPU
+baseline leg import this package; the product (``decode_context_attention_dcp_b200``)
+never does.  The arithmetic lives in ``dcp_oracle.c`` (plain C loops in double
+precision, built here with gcc -O2 -fno-fast-math); this module only compiles
+it and marshals numpy arrays in and out.
+
+Sources, by page and section:
+  * vLLM API docs, ``vllm.v1.attention.ops.dcp_alltoall``: ``_lse_weighted_combine``
+    (the combine) and ``dcp_a2a_lse_reduce`` (the packed [N, B, H/N, D+pack] layout).
+  * vllm-ascend ``attention/context_parallel/sfa_cp.py``: ``_merge_dcp_outputs_with_torch``
+    (the softmax form of the merge) and ``_get_dcp_local_seq_lens`` (interleaved KV shards).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "dcp_oracle.c")
+LIBRARY = os.path.join(_HERE, "liboracle.so")
+
+# The oracle's own dtype codes (see dcp_oracle.c).
+BF16, FP16, FP32, F64 = 0, 1, 2, 3
+
+_c_i64 = ctypes.c_int64
+_c_int = ctypes.c_int
+_c_ptr = ctypes.c_void_p
+
+
+def compile_oracle(source: str = SOURCE, output: str = LIBRARY) -> str:
+    """Compile the C oracle into a shared library (atomically replaces ``output``)."""
+    fd, tmp = tempfile.mkstemp(suffix=".so", dir=os.path.dirname(output))
+    os.close(fd)
+    try:
+        subprocess.run(
+            ["gcc", "-O2", "-fno-fast-math", "-std=c11", "-fPIC", "-shared", "-o", tmp, source, "-lm"],
+            check=True,
+        )
+        os.replace(tmp, output)
+    finally:
+        if os.path.exists(tmp):
+            os.unlink(tmp)
+    return output
+
+
+def _stale(lib: str, src: str) -> bool:
+    return not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src)
+
+
+class Oracle:
+    """ctypes view of one build of ``dcp_oracle.c``."""
+
+    def __init__(self, library: str):
+        self.path = library
+        lib = ctypes.CDLL(library)
+        lib.oracle_lse_pack_dim.argtypes = [_c_int]
+        lib.oracle_lse_pack_dim.restype = _c_int
+        lib.oracle_decode.argtypes = [_c_ptr, _c_int, _c_i64]
+        lib.oracle_decode.restype = ctypes.c_double
+        lib.oracle_pack.argtypes = [_c_ptr, _c_ptr, _c_ptr, _c_i64, _c_i64, _c_i64, _c_int, _c_int,
+                                    _c_i64, _c_i64, _c_i64]
+        lib.oracle_pack.restype = _c_int
+        lib.oracle_unpack.argtypes = [_c_ptr, _c_ptr, _c_ptr, _c_int, _c_i64, _c_i64, _c_i64, _c_i64, _c_int]
+        lib.oracle_unpack.restype = _c_int
+        lib.oracle_lse_combine.argtypes = [_c_ptr, _c_int, _c_ptr, _c_int, _c_ptr, _c_ptr, _c_int,
+                                           _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_int]
+        lib.oracle_lse_combine.restype = _c_int
+        lib.oracle_unpack_combine.argtypes = [_c_ptr, _c_int, _c_ptr, _c_ptr, _c_int, _c_i64, _c_i64,
+                                              _c_i64, _c_i64, _c_int, _c_int]
+        lib.oracle_unpack_combine.restype = _c_int
+        lib.oracle_softmax_merge.argtypes = [_c_ptr, _c_int, _c_ptr, _c_int, _c_ptr, _c_int, _c_i64,
+                                             _c_i64, _c_i64, _c_i64, _c_i64]
+        lib.oracle_softmax_merge.restype = _c_int
+        lib.oracle_attention.argtypes = [_c_ptr, _c_ptr, _c_ptr, _c_int, _c_ptr, _c_ptr, _c_i64, _c_i64,
+                                         _c_ptr, _c_i64, ctypes.c_double, _c_int]
+        lib.oracle_attention.restype = _c_int
+        lib.oracle_local_seq_len.argtypes = [_c_i64, _c_i64, _c_i64, _c_i64]
+        lib.oracle_local_seq_len.restype = _c_i64
+        self.lib = lib
+
+    # ---- helpers -------------------------------------------------------------------
+    @staticmethod
+    def _ptr(a: np.ndarray) -> int:
+        return a.ctypes.data
+
+    @staticmethod
+    def _check(rc: int, what: str) -> None:
+        if rc != 0:
+            raise ValueError(f"oracle {what} rejected its arguments")
+
+    # ---- API -----------------------------------------------------------------------
+    def lse_pack_dim(self, dtype: int) -> int:
+        return self.lib.oracle_lse_pack_dim(dtype)
+
+    def decode(self, raw: np.ndarray, dtype: int) -> np.ndarray:
+        """Decode raw element bits (uint16 for bf16/fp16) to float64, element by element."""
+        raw = np.ascontiguousarray(raw)
+        flat = raw.reshape(-1)
+        out = np.empty(flat.shape[0], dtype=np.float64)
+        for i in range(flat.shape[0]):
+            out[i] = self.lib.oracle_decode(self._ptr(flat), dtype, i)
+        return out.reshape(raw.shape)
+
+    def pack(self, cp_attn_out: np.ndarray, cp_attn_lse: np.ndarray, world_size: int, dtype: int,
+             out_strides: tuple[int, int] | None = None, lse_stride_b: int | None = None) -> np.ndarray:
+        """cp_attn_out [B, H, D] raw elements (uint16 / float32), cp_attn_lse [B, H] float32 ->
+        send buffer [world_size, B, H/world_size, D + pack] of raw elements."""
+        B, H, D = cp_attn_out.shape
+        es = cp_attn_out.dtype.itemsize
+        if out_strides is None:
+            out_strides = (cp_attn_out.strides[0] // es, cp_attn_out.strides[1] // es)
+        if lse_stride_b is None:
+            lse_stride_b = cp_attn_lse.strides[0] // 4
+        assert cp_attn_out.strides[2] == es and cp_attn_lse.strides[1] == 4
+        pack = self.lse_pack_dim(dtype)
+        send = np.zeros((world_size, B, H // max(world_size, 1), D + pack), dtype=cp_attn_out.dtype)
+        rc = self.lib.oracle_pack(self._ptr(cp_attn_out), self._ptr(cp_attn_lse), self._ptr(send), B, H, D,
+                                  world_size, dtype, out_strides[0], out_strides[1], lse_stride_b)
+        self._check(rc, "pack")
+        return send
+
+    def unpack(self, recv: np.ndarray, dtype: int, D: int) -> tuple[np.ndarray, np.ndarray]:
+        N, B, Hr, W = recv.shape
+        recv = np.ascontiguousarray(recv)
+        outs = np.zeros((N, B, Hr, D), dtype=recv.dtype)
+        lses = np.zeros((N, B, Hr), dtype=np.float32)
+        rc = self.lib.oracle_unpack(self._ptr(recv), self._ptr(outs), self._ptr(lses), N, B, Hr, D,
+                                    B * Hr * W, dtype)
+        self._check(rc, "unpack")
+        return outs, lses
+
+    def lse_combine(self, outputs: np.ndarray, out_dtype: int, lses: np.ndarray, return_lse: bool = False,
+                    is_lse_base_on_e: bool = True):
+        """outputs [N, B, H, D] raw elements (or float64 with out_dtype=F64), lses [N, B, H]
+        float32 or float64 -> result [B, H, D] float64 (+ global LSE [B, H] float64)."""
+        outputs = np.ascontiguousarray(outputs)
+        lses = np.ascontiguousarray(lses)
+        N, B, H, D = outputs.shape
+        assert lses.shape == (N, B, H)
+        lse_dtype = F64 if lses.dtype == np.float64 else FP32
+        assert lses.dtype in (np.float32, np.float64)
+        result = np.zeros((B, H, D), dtype=np.float64)
+        glse = np.zeros((B, H), dtype=np.float64)
+        rc = self.lib.oracle_lse_combine(self._ptr(outputs), out_dtype, self._ptr(lses), lse_dtype,
+                                         self._ptr(result), self._ptr(glse), N, B, H, D, B * H * D, B * H,
+                                         int(is_lse_base_on_e), int(return_lse))
+        self._check(rc, "lse_combine")
+        return (result, glse) if return_lse else result
+
+    def lse_combine_rows(self, outputs: np.ndarray, out_dtype: int, lses: np.ndarray, rows,
+                         return_lse: bool = False, is_lse_base_on_e: bool = True):
+        """The combine of selected (b, h) rows only, read in place from full-size arrays.
+
+        outputs [N, B, H, D] / lses [N, B, H] must be C-contiguous; ``rows`` is a list of (b, h).
+        Returns ([len(rows), D] float64, [len(rows)] float64)."""
+        assert outputs.flags.c_contiguous and lses.flags.c_contiguous
+        N, B, H, D = outputs.shape
+        lse_dtype = F64 if lses.dtype == np.float64 else FP32
+        es, ls = outputs.dtype.itemsize, lses.dtype.itemsize
+        res = np.zeros((len(rows), D), dtype=np.float64)
+        gl = np.zeros(len(rows), dtype=np.float64)
+        for i, (b, h) in enumerate(rows):
+            unit = b * H + h
+            rc = self.lib.oracle_lse_combine(self._ptr(outputs) + unit * D * es, out_dtype,
+                                             self._ptr(lses) + unit * ls, lse_dtype,
+                                             self._ptr(res) + i * D * 8, self._ptr(gl) + i * 8,
+                                             N, 1, 1, D, B * H * D, B * H, int(is_lse_base_on_e), int(return_lse))
+            self._check(rc, "lse_combine")
+        return res, gl
+
+    def unpack_combine(self, recv: np.ndarray, dtype: int, D: int, return_lse: bool = False,
+                       is_lse_base_on_e: bool = True):
+        recv = np.ascontiguousarray(recv)
+        N, B, Hr, W = recv.shape
+        result = np.zeros((B, Hr, D), dtype=np.float64)
+        glse = np.zeros((B, Hr), dtype=np.float64)
+        rc = self.lib.oracle_unpack_combine(self._ptr(recv), dtype, self._ptr(result), self._ptr(glse), N, B, Hr,
+                                            D, B * Hr * W, int(is_lse_base_on_e), int(return_lse))
+        self._check(rc, "unpack_combine")
+        return (result, glse) if return_lse else result
+
+    def unpack_combine_rows(self, recv: np.ndarray, dtype: int, D: int, rows, return_lse: bool = False,
+                            is_lse_base_on_e: bool = True):
+        """unpack+combine of selected (b, h) rows, read in place from a C-contiguous [N, B, Hr, W] buffer."""
+        assert recv.flags.c_contiguous
+        N, B, Hr, W = recv.shape
+        es = recv.dtype.itemsize
+        res = np.zeros((len(rows), D), dtype=np.float64)
+        gl = np.zeros(len(rows), dtype=np.float64)
+        for i, (b, h) in enumerate(rows):
+            unit = b * Hr + h
+            rc = self.lib.oracle_unpack_combine(self._ptr(recv) + unit * W * es, dtype, self._ptr(res) + i * D * 8,
+                                                self._ptr(gl) + i * 8, N, 1, 1, D, B * Hr * W,
+                                                int(is_lse_base_on_e), int(return_lse))
+            self._check(rc, "unpack_combine")
+        return res, gl
+
+    def softmax_merge(self, outputs: np.ndarray, out_dtype: int, lses: np.ndarray) -> np.ndarray:
+        outputs = np.ascontiguousarray(outputs)
+        lses = np.ascontiguousarray(lses)
+        N, B, H, D = outputs.shape
+        lse_dtype = F64 if lses.dtype == np.float64 else FP32
+        result = np.zeros((B, H, D), dtype=np.float64)
+        rc = self.lib.oracle_softmax_merge(self._ptr(outputs), out_dtype, self._ptr(lses), lse_dtype,
+                                           self._ptr(result), N, B, H, D, B * H * D, B * H)
+        self._check(rc, "softmax_merge")
+        return result
+
+    def attention(self, q: np.ndarray, k: np.ndarray, v: np.ndarray, dtype: int, positions,
+                  scale: float, is_lse_base_on_e: bool = True) -> tuple[np.ndarray, np.ndarray]:
+        """One token: q [H, D], k/v [L, H, D] -> (out [H, D] f64, lse [H] f64) over ``positions``."""
+        q, k, v = (np.ascontiguousarray(x) for x in (q, k, v))
+        H, D = q.shape
+        pos = np.ascontiguousarray(np.asarray(positions, dtype=np.int64))
+        out = np.zeros((H, D), dtype=np.float64)
+        lse = np.zeros(H, dtype=np.float64)
+        rc = self.lib.oracle_attention(self._ptr(q), self._ptr(k), self._ptr(v), dtype, self._ptr(out),
+                                       self._ptr(lse), H, D, self._ptr(pos) if len(pos) else None, len(pos),
+                                       float(scale), int(is_lse_base_on_e))
+        self._check(rc, "attention")
+        return out, lse
+
+    def local_seq_len(self, seq_len: int, cp_size: int, rank: int, interleave: int) -> int:
+        return self.lib.oracle_local_seq_len(seq_len, cp_size, rank, interleave)
+
+
+_default: Oracle | None = None
+
+
+def load() -> Oracle:
+    """The oracle built from ``dcp_oracle.c`` (compiled on first use or when the source changed)."""
+    global _default
+    if _default is None:
+        if _stale(LIBRARY, SOURCE):
+            compile_oracle()
+        _default = Oracle(LIBRARY)
+    return _default
