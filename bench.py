@@ -1,0 +1,419 @@
+#!/usr/bin/env python3
+"""Bench of the DCP combine hot path on B200: one step = dcp_pack + dcp_unpack_combine.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole path over one batch: the pack of one rank's partial
+attention output cp_attn_out [B, N*Hr, D] (+ LSE [B, N*Hr]) into the packed buffer
+[N, B, Hr, D+2], then the fused unpack+combine of that buffer (every shard taken from it)
+into [B, Hr, D].  Default workload: the largest bandwidth-sweep point (N=16, B=16384,
+Hr=16, D=512, bf16).  Inputs are resident in HBM before timing and larger than L2.
+
+Metric: effective HBM GB/s = algorithmic bytes / device time (CUDA events on the launching
+stream), max over ranks; also (token*head)/s and the fraction of the measured HBM peak.
+With N > 1 (torchrun, one process per GPU) every rank combines its own batch: weak scaling,
+no data-path collective.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded sample of the same
+workload (rank 0 only), for the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "combine effective HBM GB/s and fraction of B200 peak; (token·head)/s"
+DEFAULT_WORKLOAD = "sweep_N16_B16384_D512"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---- multi-process plumbing (testable on CPU with gloo) -----------------------------------
+def dist_env() -> tuple[int, int, int]:
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Weak scaling: every rank combines its own batch of the same shape, drawn with its own seed."""
+    return base_seed + 7919 * rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None) -> None:
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---- measurement side data -----------------------------------------------------------------
+def kernel_digest() -> str:
+    """Hash of the kernel sources: ncu counters are reported only for the code they were taken on."""
+    h = hashlib.sha256()
+    for sub in ("decode_context_attention_dcp_b200/csrc", "include"):
+        d = os.path.join(ROOT, sub)
+        for name in sorted(os.listdir(d)):
+            with open(os.path.join(d, name), "rb") as fh:
+                h.update(name.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peak() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            v = float(json.load(fh)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_traffic(kernel: str, workload: str) -> float | None:
+    """DRAM bytes per launch (read + write) from the committed ncu summary, if it was taken on the
+    current kernel sources.  Table rows: | kernel | workload | digest | dram_read | dram_write | ..."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    if not os.path.exists(path):
+        return None
+    digest = kernel_digest()
+    for line in open(path):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 5 and cells[0] == kernel and cells[1] == workload and cells[2] == digest:
+            try:
+                return float(cells[3]) + float(cells[4])
+            except ValueError:
+                return None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU works."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu=timestamp,{self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            c = [x.strip() for x in line.split(",")]
+            if len(c) < 9:
+                continue
+            try:
+                rows.append((float(c[1]), float(c[2]), c[4:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        max_mhz = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[0] >= 0.5 * max_mhz] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2][1:]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max_mhz, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---- the CPU oracle (reference arm and CPU baseline) -----------------------------------------
+def oracle_step_sample(w, tokens: int):
+    """One oracle step (pack + unpack+combine, plain fp64 C) on the first ``tokens`` tokens of the
+    workload's rank-0 inputs.  Returns (seconds, algorithmic bytes)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from decode_context_attention_dcp_b200 import workloads as wl
+
+    ws = w.with_(B=tokens)
+    cp_out, cp_lse = wl.pack_inputs(ws)
+    o = oracle.load()
+    code = {torch.bfloat16: oracle.BF16, torch.float16: oracle.FP16, torch.float32: oracle.FP32}[cp_out.dtype]
+    ro = cp_out.view(torch.int16).numpy().view(np.uint16) if cp_out.element_size() == 2 else cp_out.numpy()
+    t0 = time.perf_counter()
+    send = o.pack(ro, cp_lse.numpy(), ws.N, code)
+    o.unpack_combine(send, code, ws.D, return_lse=ws.return_lse, is_lse_base_on_e=ws.is_lse_base_on_e)
+    dt = time.perf_counter() - t0
+    return dt, ws.pack_bytes() + ws.combine_bytes()
+
+
+def cpu_baseline(w, budget_s: float = 12.0) -> dict:
+    tokens = max(1, w.B // 8)
+    total_t, total_b, reps = 0.0, 0, 0
+    while total_t < budget_s and reps < 8:
+        dt, nb = oracle_step_sample(w, tokens)
+        total_t += dt
+        total_b += nb
+        reps += 1
+    return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{reps} x (pack + unpack_combine) of the first {tokens} of {w.B} tokens, "
+                      f"single-threaded fp64 C, {total_t:.1f} s"}
+
+
+def run_reference(args) -> int:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from decode_context_attention_dcp_b200 import workloads as wl
+
+    w = wl.by_name(args.workload)
+    tokens = max(1, min(w.B, 256))
+    for _ in range(args.warmup):
+        oracle_step_sample(w, tokens)
+    secs, nbytes = 0.0, 0
+    for _ in range(args.steps):
+        dt, nb = oracle_step_sample(w, tokens)
+        secs += dt
+        nbytes += nb
+    gbs = nbytes / secs / 1e9
+    sample = f"each step: pack + unpack_combine of the first {tokens} of {w.B} tokens, single-threaded fp64 C"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w) -> dict:
+    return {"workload": w.name, "step": "dcp_pack + dcp_unpack_combine", "shards": w.N, "tokens": w.B,
+            "heads_in": w.H, "heads_out": w.Hr, "head_dim": w.D, "io_dtype": w.dtype,
+            "is_lse_base_on_e": w.is_lse_base_on_e, "return_lse": w.return_lse,
+            "lse": f"U[{w.lse_lo},{w.lse_hi}], {w.p_neginf:.0%} -inf",
+            "l2": "inputs larger than L2 (no flush between steps)"}
+
+
+# ---- our arm ---------------------------------------------------------------------------------
+def run_ours(args) -> int:
+    import torch
+    import torch.distributed as dist
+
+    import decode_context_attention_dcp_b200 as dcp
+    from decode_context_attention_dcp_b200 import workloads as wl
+
+    rank, world, local_rank = dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    lib = dcp.library()
+
+    w = wl.by_name(args.workload)
+    wr = w.with_(seed=rank_seed(w.seed, rank))
+    cp_out_h, cp_lse_h = wl.pack_inputs(wr, pin_memory=True)
+    cp_out = cp_out_h.to(device)
+    cp_lse = cp_lse_h.to(device)
+    P = dcp.dcp_lse_pack_dim(cp_out.dtype)
+    send = torch.empty((w.N, w.B, w.Hr, w.D + P), dtype=cp_out.dtype, device=device)
+    result = torch.empty((w.B, w.Hr, w.D), dtype=cp_out.dtype, device=device)
+    glse = torch.empty((w.B, w.Hr), dtype=torch.float32, device=device) if w.return_lse else None
+    stream = torch.cuda.Stream(device)
+    sh = stream.cuda_stream
+    code = dcp.DTYPE_CODES[cp_out.dtype]
+    glse_ptr = glse.data_ptr() if glse is not None else None
+
+    def pack(src, lse):
+        st = lib.dcp_pack(src.data_ptr(), lse.data_ptr(), send.data_ptr(), w.B, w.H, w.D, w.N, code,
+                          src.stride(0), src.stride(1), lse.stride(0), sh)
+        if st:
+            raise dcp.DCPError(st, dcp.dcp_last_error())
+
+    def combine():
+        st = lib.dcp_unpack_combine(send.data_ptr(), result.data_ptr(), glse_ptr, w.N, w.B, w.Hr, w.D,
+                                    send.stride(0), code, int(w.is_lse_base_on_e), int(w.return_lse), sh)
+        if st:
+            raise dcp.DCPError(st, dcp.dcp_last_error())
+
+    K, W = args.steps, args.warmup
+    torch.cuda.synchronize(device)
+    clocks = None
+    sampler = None
+    if not args.no_clocks:
+        uuid = getattr(torch.cuda.get_device_properties(device), "uuid", None)
+        sampler = ClockSampler(f"GPU-{uuid}" if uuid else None)
+        sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(W):
+            pack(cp_out, cp_lse)
+            combine()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * K + 1)]
+        stream.synchronize()
+        barrier(device)
+        torch.cuda.synchronize(device)
+        ev[0].record(stream)
+        for k in range(K):
+            pack(cp_out, cp_lse)
+            ev[3 * k + 1].record(stream)
+            combine()
+            ev[3 * k + 2].record(stream)
+            if k + 1 < K:
+                ev[3 * k + 3].record(stream)
+        ev[3 * K].record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    if sampler is not None:
+        clocks = sampler.stop()
+    # per-kernel device time over the timed region: pack = [start of step, after pack],
+    # combine = [after pack, after combine]
+    t_pack = sum((ev[0] if k == 0 else ev[3 * k]).elapsed_time(ev[3 * k + 1]) for k in range(K))
+    t_comb = sum(ev[3 * k + 1].elapsed_time(ev[3 * k + 2]) for k in range(K))
+    t_total = ev[0].elapsed_time(ev[3 * K])
+    t_total_max = max_over_ranks(t_total, device)
+    t_pack_max = max_over_ranks(t_pack, device)
+    t_comb_max = max_over_ranks(t_comb, device)
+
+    bytes_pack, bytes_comb = w.pack_bytes(), w.combine_bytes()
+    step_bytes = bytes_pack + bytes_comb
+    ms_per_step = t_total_max / K
+    value = world * step_bytes * K / (t_total_max * 1e-3) / 1e9
+    peak, peak_src = load_peak()
+    kernels = {
+        "dcp_pack": {"ms_per_launch": t_pack_max / K, "bytes_per_launch": bytes_pack,
+                     "gbs": bytes_pack / (t_pack_max / K * 1e-3) / 1e9},
+        "dcp_unpack_combine": {"ms_per_launch": t_comb_max / K, "bytes_per_launch": bytes_comb,
+                               "gbs": bytes_comb / (t_comb_max / K * 1e-3) / 1e9},
+    }
+    for v in kernels.values():
+        v["frac_of_peak"] = v["gbs"] / peak
+        v["share_of_step"] = v["ms_per_launch"] / ms_per_step
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"])
+    dk = kernels[dom]
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": dk["gbs"], "peak": peak, "unit": "GB/s",
+                "frac": dk["gbs"] / peak, "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json hbm_gbs' if peak_src == 'measured' else 'profiling recipe fallback'})",
+                "traffic": load_traffic(dom, w.name), "algorithmic_bytes_per_launch": dk["bytes_per_launch"]}
+
+    # end to end through the public API: pinned host inputs in, host result out, every step
+    e2e = None
+    if not args.no_e2e:
+        res_h = torch.empty(result.shape, dtype=result.dtype, pin_memory=True)
+        glse_h = torch.empty(glse.shape, dtype=glse.dtype, pin_memory=True) if glse is not None else None
+        d_out = torch.empty_like(cp_out)
+        d_lse = torch.empty_like(cp_lse)
+
+        def e2e_step():
+            d_out.copy_(cp_out_h, non_blocking=True)
+            d_lse.copy_(cp_lse_h, non_blocking=True)
+            dcp.dcp_pack(d_out, d_lse, send, w.N)
+            dcp.dcp_unpack_combine(send, result, glse, is_lse_base_on_e=w.is_lse_base_on_e,
+                                   return_lse=w.return_lse)
+            res_h.copy_(result, non_blocking=True)
+            if glse_h is not None:
+                glse_h.copy_(glse, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            e2e_step()
+            stream.synchronize()
+            barrier(device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.e2e_steps):
+                e2e_step()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+        t_e2e = max_over_ranks(e0.elapsed_time(e1), device)
+        h2d = cp_out.numel() * cp_out.element_size() + cp_lse.numel() * 4
+        d2h = result.numel() * result.element_size() + (glse.numel() * 4 if glse is not None else 0)
+        e2e = {"value": world * step_bytes * args.e2e_steps / (t_e2e * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "ms_per_step": t_e2e / args.e2e_steps}
+        del d_out, d_lse
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic", "config": workload_config(w),
+            "token_heads_per_s": world * w.B * w.Hr * K / (t_total_max * 1e-3),
+            "frac_of_measured_peak": value / peak, "frac_of_nominal_8tbs": value / NOMINAL_HBM_GBS,
+            "kernels": kernels, "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu,
+            "gpu_launches": 2 * K, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier(device)
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None) -> int:
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,230 @@
+"""B200 (sm_100a) DCP LSE-weighted combine: thin Python binding of libdcpcombine.so.
+
+The three device steps of the decode-context-parallel combine (vLLM API docs,
+vllm.v1.attention.ops.dcp_alltoall: _lse_weighted_combine and
+dcp_a2a_lse_reduce) run in hand-written CUDA kernels behind a C ABI
+(include/dcp_combine.h).  This module only marshals torch CUDA tensors into
+pointers, sizes, strides and the current stream; every step of the
+computation happens in the library.  There is no fallback: if the library
+cannot be built or loaded, every call raises.
+
+Low-level calls (same names as the C ABI, caller-allocated outputs):
+    dcp_pack(cp_attn_out, cp_attn_lse, send_buf, world_size)
+    dcp_lse_combine(outputs, lses, result, global_lse=None, ...)
+    dcp_unpack_combine(recv_buf, result, global_lse=None, ...)
+    dcp_lse_pack_dim(dtype), dcp_last_error()
+
+Allocating helpers with the pages' argument conventions:
+    lse_weighted_combine(outputs, lses, return_lse=False, is_lse_base_on_e=True)
+    pack(cp_attn_out, cp_attn_lse, world_size)
+    unpack_combine(recv_buf, return_lse=False, is_lse_base_on_e=True)
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+
+import torch
+
+from . import _build
+
+__all__ = [
+    "DCPError", "library", "dcp_lse_pack_dim", "dcp_pack", "dcp_lse_combine", "dcp_unpack_combine",
+    "dcp_last_error", "dcp_version", "lse_weighted_combine", "pack", "unpack_combine", "DTYPE_CODES",
+]
+
+DTYPE_CODES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
+STATUS_NAMES = {0: "DCP_OK", 1: "DCP_ERR_INVALID_ARG", 2: "DCP_ERR_UNSUPPORTED_DTYPE", 3: "DCP_ERR_MISALIGNED",
+                4: "DCP_ERR_SHAPE", 5: "DCP_ERR_CUDA"}
+
+_i32, _i64, _ptr = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p
+_lib: ctypes.CDLL | None = None
+_lock = threading.Lock()
+
+
+class DCPError(RuntimeError):
+    """A non-OK status from libdcpcombine.so (``status`` holds the dcp_status code)."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def library() -> ctypes.CDLL:
+    """The loaded C library (built in-tree first if it is missing or older than its sources)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                path = _build.build()
+                lib = ctypes.CDLL(path)
+                lib.dcp_lse_pack_dim.argtypes = [_i32]
+                lib.dcp_lse_pack_dim.restype = _i32
+                lib.dcp_pack.argtypes = [_ptr, _ptr, _ptr, _i64, _i64, _i64, _i32, _i32, _i64, _i64, _i64, _ptr]
+                lib.dcp_pack.restype = _i32
+                lib.dcp_lse_combine.argtypes = [_ptr, _ptr, _ptr, _ptr, _i32, _i64, _i64, _i64, _i64, _i64, _i32,
+                                                _i32, _i32, _ptr]
+                lib.dcp_lse_combine.restype = _i32
+                lib.dcp_unpack_combine.argtypes = [_ptr, _ptr, _ptr, _i32, _i64, _i64, _i64, _i64, _i32, _i32, _i32,
+                                                   _ptr]
+                lib.dcp_unpack_combine.restype = _i32
+                lib.dcp_last_error.argtypes = []
+                lib.dcp_last_error.restype = ctypes.c_char_p
+                lib.dcp_version.argtypes = []
+                lib.dcp_version.restype = _i32
+                _lib = lib
+    return _lib
+
+
+def dcp_last_error() -> str:
+    return library().dcp_last_error().decode()
+
+
+def dcp_version() -> int:
+    return library().dcp_version()
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise DCPError(status, dcp_last_error())
+
+
+def _code(dtype: torch.dtype) -> int:
+    if dtype not in DTYPE_CODES:
+        raise DCPError(2, f"unsupported dtype {dtype}")
+    return DTYPE_CODES[dtype]
+
+
+def _cuda(*tensors: torch.Tensor | None) -> torch.device:
+    dev = None
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("all tensors must be on the same device")
+    return dev
+
+
+def _stream(device: torch.device, stream) -> int:
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return s.cuda_stream if isinstance(s, torch.cuda.Stream) else int(s)
+
+
+def _inner_contiguous(t: torch.Tensor, dims: int, what: str) -> None:
+    """The last ``dims`` dimensions of ``t`` must be laid out contiguously."""
+    expect = 1
+    for d in range(t.dim() - 1, t.dim() - 1 - dims, -1):
+        if t.size(d) != 1 and t.stride(d) != expect:
+            raise ValueError(f"{what}: the last {dims} dimensions must be contiguous (strides {t.stride()})")
+        expect *= t.size(d)
+
+
+def dcp_lse_pack_dim(dtype: torch.dtype) -> int:
+    """Output-dtype slots that carry one fp32 LSE in a packed row (2 for bf16/fp16, 1 for fp32)."""
+    return library().dcp_lse_pack_dim(_code(dtype))
+
+
+def dcp_pack(cp_attn_out: torch.Tensor, cp_attn_lse: torch.Tensor, send_buf: torch.Tensor, world_size: int,
+             stream=None) -> None:
+    """cp_attn_out [B, H, D] + cp_attn_lse [B, H] fp32 -> send_buf [world_size, B, H/world_size, D + P]."""
+    dev = _cuda(cp_attn_out, cp_attn_lse, send_buf)
+    B, H, D = cp_attn_out.shape
+    if cp_attn_lse.shape != (B, H) or cp_attn_lse.dtype != torch.float32:
+        raise ValueError(f"cp_attn_lse must be fp32 [{B}, {H}], got {cp_attn_lse.dtype} {tuple(cp_attn_lse.shape)}")
+    if cp_attn_out.stride(2) != 1 or cp_attn_lse.stride(1) != 1:
+        raise ValueError("cp_attn_out and cp_attn_lse must be contiguous in their last dimension")
+    if send_buf.dtype != cp_attn_out.dtype or not send_buf.is_contiguous():
+        raise ValueError("send_buf must be contiguous and of the output dtype")
+    code = _code(cp_attn_out.dtype)
+    lib = library()
+    P = lib.dcp_lse_pack_dim(code)
+    if world_size >= 1 and H % world_size == 0 and send_buf.shape != (world_size, B, H // world_size, D + P):
+        raise ValueError(f"send_buf must have shape {(world_size, B, H // world_size, D + P)}")
+    with torch.cuda.device(dev):
+        _check(lib.dcp_pack(cp_attn_out.data_ptr(), cp_attn_lse.data_ptr(), send_buf.data_ptr(), B, H, D,
+                            int(world_size), code, cp_attn_out.stride(0), cp_attn_out.stride(1),
+                            cp_attn_lse.stride(0), _stream(dev, stream)))
+
+
+def dcp_lse_combine(outputs: torch.Tensor, lses: torch.Tensor, result: torch.Tensor,
+                    global_lse: torch.Tensor | None = None, is_lse_base_on_e: bool = True,
+                    return_lse: bool = False, stream=None) -> None:
+    """outputs [N, B, H, D] + lses [N, B, H] fp32 -> result [B, H, D] (+ global_lse [B, H] fp32).
+
+    dim 0 of outputs / lses may have any stride (a capacity-strided receive buffer); the rest
+    must be contiguous."""
+    dev = _cuda(outputs, lses, result, global_lse)
+    N, B, H, D = outputs.shape
+    if lses.shape != (N, B, H) or lses.dtype != torch.float32:
+        raise ValueError(f"lses must be fp32 [{N}, {B}, {H}], got {lses.dtype} {tuple(lses.shape)}")
+    _inner_contiguous(outputs, 3, "outputs")
+    _inner_contiguous(lses, 2, "lses")
+    if result.shape != (B, H, D) or result.dtype != outputs.dtype or not result.is_contiguous():
+        raise ValueError("result must be a contiguous [B, H, D] tensor of the output dtype")
+    if return_lse and (global_lse is None or global_lse.shape != (B, H) or global_lse.dtype != torch.float32
+                       or not global_lse.is_contiguous()):
+        raise ValueError("return_lse needs a contiguous fp32 [B, H] global_lse")
+    with torch.cuda.device(dev):
+        _check(library().dcp_lse_combine(
+            outputs.data_ptr(), lses.data_ptr(), result.data_ptr(),
+            global_lse.data_ptr() if (return_lse and global_lse is not None) else None,
+            N, B, H, D, outputs.stride(0) if N > 1 else B * H * D, lses.stride(0) if N > 1 else B * H,
+            _code(outputs.dtype), int(bool(is_lse_base_on_e)), int(bool(return_lse)), _stream(dev, stream)))
+
+
+def dcp_unpack_combine(recv_buf: torch.Tensor, result: torch.Tensor, global_lse: torch.Tensor | None = None,
+                       is_lse_base_on_e: bool = True, return_lse: bool = False, stream=None) -> None:
+    """recv_buf [N, B, Hr, D + P] -> result [B, Hr, D] (+ global_lse [B, Hr] fp32)."""
+    dev = _cuda(recv_buf, result, global_lse)
+    N, B, Hr, W = recv_buf.shape
+    code = _code(recv_buf.dtype)
+    D = W - library().dcp_lse_pack_dim(code)
+    _inner_contiguous(recv_buf, 3, "recv_buf")
+    if result.shape != (B, Hr, D) or result.dtype != recv_buf.dtype or not result.is_contiguous():
+        raise ValueError(f"result must be a contiguous [{B}, {Hr}, {D}] tensor of the buffer dtype")
+    if return_lse and (global_lse is None or global_lse.shape != (B, Hr) or global_lse.dtype != torch.float32
+                       or not global_lse.is_contiguous()):
+        raise ValueError("return_lse needs a contiguous fp32 [B, Hr] global_lse")
+    with torch.cuda.device(dev):
+        _check(library().dcp_unpack_combine(
+            recv_buf.data_ptr(), result.data_ptr(),
+            global_lse.data_ptr() if (return_lse and global_lse is not None) else None,
+            N, B, Hr, D, recv_buf.stride(0) if N > 1 else B * Hr * W, code, int(bool(is_lse_base_on_e)),
+            int(bool(return_lse)), _stream(dev, stream)))
+
+
+# ---- allocating helpers ------------------------------------------------------------------
+def lse_weighted_combine(outputs: torch.Tensor, lses: torch.Tensor, return_lse: bool = False,
+                         is_lse_base_on_e: bool = True):
+    """Same arguments and results as the pages' _lse_weighted_combine, computed on the GPU:
+    outputs [N, B, H, D], lses [N, B, H] -> [B, H, D] (and the global LSE [B, H] fp32)."""
+    N, B, H, D = outputs.shape
+    result = torch.empty((B, H, D), dtype=outputs.dtype, device=outputs.device)
+    glse = torch.empty((B, H), dtype=torch.float32, device=outputs.device) if return_lse else None
+    dcp_lse_combine(outputs, lses, result, glse, is_lse_base_on_e=is_lse_base_on_e, return_lse=return_lse)
+    return (result, glse) if return_lse else result
+
+
+def pack(cp_attn_out: torch.Tensor, cp_attn_lse: torch.Tensor, world_size: int) -> torch.Tensor:
+    """The packed send buffer [world_size, B, H/world_size, D + P] of cp_attn_out / cp_attn_lse."""
+    B, H, D = cp_attn_out.shape
+    if world_size < 1 or H % world_size != 0:
+        raise ValueError(f"H={H} heads do not split evenly over {world_size} ranks")
+    P = dcp_lse_pack_dim(cp_attn_out.dtype)
+    send = torch.empty((world_size, B, H // world_size, D + P), dtype=cp_attn_out.dtype, device=cp_attn_out.device)
+    dcp_pack(cp_attn_out, cp_attn_lse, send, world_size)
+    return send
+
+
+def unpack_combine(recv_buf: torch.Tensor, return_lse: bool = False, is_lse_base_on_e: bool = True):
+    """Combine of a packed receive buffer [N, B, Hr, D + P] -> [B, Hr, D] (and [B, Hr] fp32)."""
+    N, B, Hr, W = recv_buf.shape
+    D = W - dcp_lse_pack_dim(recv_buf.dtype)
+    result = torch.empty((B, Hr, D), dtype=recv_buf.dtype, device=recv_buf.device)
+    glse = torch.empty((B, Hr), dtype=torch.float32, device=recv_buf.device) if return_lse else None
+    dcp_unpack_combine(recv_buf, result, glse, is_lse_base_on_e=is_lse_base_on_e, return_lse=return_lse)
+    return (result, glse) if return_lse else result

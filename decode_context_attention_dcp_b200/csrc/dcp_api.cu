@@ -1,0 +1,288 @@
+// dcp_api.cu -- the extern "C" entry points of libdcpcombine.so (see
+// include/dcp_combine.h for the contract of each call).
+//
+// Host side only: argument validation (before any CUDA call), choice of the
+// kernel instance for the row width, grid sizing, launch, and launch-error
+// reporting.  Nothing here allocates device memory or synchronises.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <atomic>
+
+#include "dcp_combine.h"
+#include "dcp_kernels.cuh"
+
+namespace {
+
+thread_local char g_error[512] = "";
+
+int32_t fail(int32_t status, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_error, sizeof g_error, fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int32_t ok() {
+    g_error[0] = '\0';
+    return DCP_OK;
+}
+
+int elem_size(int32_t dtype) {
+    switch (dtype) {
+        case DCP_BF16:
+        case DCP_FP16: return 2;
+        case DCP_FP32: return 4;
+        default: return 0;
+    }
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+constexpr int64_t kMaxD = 8192;            // elements per row
+constexpr int64_t kMaxRows = int64_t(1) << 40;
+
+// Multiprocessor count of the current device (cached per device).
+int sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64) {
+        int v = cache[dev].load(std::memory_order_relaxed);
+        if (v > 0) return v;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+// Resident CTAs per SM of one kernel instance (cached per instance; the pool's
+// devices are identical).
+template <class K>
+int resident_ctas(K kernel, int threads, size_t smem) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess || n <= 0) n = 1;
+    return n;
+}
+
+int32_t launch_status(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(DCP_ERR_CUDA, "%s: kernel launch failed: %s", what, cudaGetErrorString(e));
+    return ok();
+}
+
+// ---------------------------------------------------------------------------
+// combine dispatch
+template <class T, int VW, int G, int CPL, int NB, bool PACKED>
+int32_t launch_combine(const dcp::CombineArgs &a, cudaStream_t stream) {
+    auto kernel = dcp::combine_kernel<T, VW, G, CPL, NB, PACKED>;
+    static const int per_sm = resident_ctas(kernel, dcp::kCombineThreads, 0);
+    constexpr int kUnitsPerWarp = 32 / G;
+    constexpr int kWarps = dcp::kCombineThreads / 32;
+    const int64_t tasks = (a.units + kUnitsPerWarp - 1) / kUnitsPerWarp;
+    const int64_t want = (tasks + kWarps - 1) / kWarps;
+    const int64_t cap = (int64_t)sm_count() * per_sm;
+    const int grid = (int)(want < cap ? want : cap);
+    kernel<<<grid, dcp::kCombineThreads, 0, stream>>>(a);
+    return launch_status(PACKED ? "dcp_unpack_combine" : "dcp_lse_combine");
+}
+
+// Lanes per row G: the smallest power of two >= the row's chunk count (at
+// least 4, at most 32).  Chunk slots per lane: ceil(chunks / G), CPL of them
+// per pass, with the loads of NB shards issued before their FMAs, so each lane
+// keeps NB * CPL * VW words in flight (32 for 16-byte chunks, 16 for words).
+template <class T, int VW, bool PACKED>
+int32_t dispatch_combine(dcp::CombineArgs a, cudaStream_t stream) {
+    const int ch = a.chunks;
+    constexpr int kSmallNB = VW == 4 ? 8 : 16;
+    if (ch <= 4) { a.slots = 1; return launch_combine<T, VW, 4, 1, kSmallNB, PACKED>(a, stream); }
+    if (ch <= 8) { a.slots = 1; return launch_combine<T, VW, 8, 1, kSmallNB, PACKED>(a, stream); }
+    if (ch <= 16) { a.slots = 1; return launch_combine<T, VW, 16, 1, kSmallNB, PACKED>(a, stream); }
+    a.slots = (ch + 31) / 32;
+    if (a.slots == 1) return launch_combine<T, VW, 32, 1, kSmallNB, PACKED>(a, stream);
+    if constexpr (VW == 4) {
+        return launch_combine<T, VW, 32, 2, 4, PACKED>(a, stream);
+    } else {
+        if (a.slots == 2) return launch_combine<T, VW, 32, 2, 8, PACKED>(a, stream);
+        if (a.slots <= 4) return launch_combine<T, VW, 32, 4, 4, PACKED>(a, stream);
+        return launch_combine<T, VW, 32, 8, 2, PACKED>(a, stream);
+    }
+}
+
+template <bool PACKED>
+int32_t dispatch_dtype(int32_t dtype, const dcp::CombineArgs &a, cudaStream_t stream) {
+    constexpr int VW = PACKED ? 1 : 4;
+    switch (dtype) {
+        case DCP_BF16: return dispatch_combine<dcp::Bf16, VW, PACKED>(a, stream);
+        case DCP_FP16: return dispatch_combine<dcp::Fp16, VW, PACKED>(a, stream);
+        default: return dispatch_combine<dcp::Fp32, VW, PACKED>(a, stream);
+    }
+}
+
+int32_t check_common(const char *fn, int32_t dtype, int32_t N, int64_t B, int64_t H, int64_t D) {
+    if (elem_size(dtype) == 0) return fail(DCP_ERR_UNSUPPORTED_DTYPE, "%s: unsupported dtype %d", fn, (int)dtype);
+    if (N < 1 || N > DCP_MAX_SHARDS)
+        return fail(DCP_ERR_INVALID_ARG, "%s: shard count %d outside [1, %d]", fn, (int)N, DCP_MAX_SHARDS);
+    if (B < 0) return fail(DCP_ERR_INVALID_ARG, "%s: negative token count %lld", fn, (long long)B);
+    if (H < 1) return fail(DCP_ERR_INVALID_ARG, "%s: head count %lld < 1", fn, (long long)H);
+    if (D < 1 || D > kMaxD) return fail(DCP_ERR_INVALID_ARG, "%s: head dim %lld outside [1, %lld]", fn, (long long)D,
+                                        (long long)kMaxD);
+    if ((D * elem_size(dtype)) % 16 != 0)
+        return fail(DCP_ERR_MISALIGNED, "%s: a row of D=%lld elements is not a multiple of 16 bytes", fn,
+                    (long long)D);
+    if (B > 0 && (B > kMaxRows / H || B * H > kMaxRows / (int64_t)N))
+        return fail(DCP_ERR_INVALID_ARG, "%s: problem too large", fn);
+    return DCP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t dcp_version(void) { return 10000; }
+
+const char *dcp_last_error(void) { return g_error; }
+
+int32_t dcp_lse_pack_dim(int32_t dtype) {
+    const int es = elem_size(dtype);
+    return es ? 4 / es : -1;
+}
+
+int32_t dcp_lse_combine(const void *outputs, const float *lses, void *result, float *global_lse, int32_t N, int64_t B,
+                        int64_t H, int64_t D, int64_t out_stride_n, int64_t lse_stride_n, int32_t dtype,
+                        int32_t is_lse_base_on_e, int32_t return_lse, void *cuda_stream) {
+    const char *fn = "dcp_lse_combine";
+    int32_t st = check_common(fn, dtype, N, B, H, D);
+    if (st != DCP_OK) return st;
+    const int es = elem_size(dtype);
+    if (out_stride_n < B * H * D)
+        return fail(DCP_ERR_INVALID_ARG, "%s: out_stride_n %lld < B*H*D = %lld", fn, (long long)out_stride_n,
+                    (long long)(B * H * D));
+    if (lse_stride_n < B * H)
+        return fail(DCP_ERR_INVALID_ARG, "%s: lse_stride_n %lld < B*H = %lld", fn, (long long)lse_stride_n,
+                    (long long)(B * H));
+    if ((out_stride_n * es) % 16 != 0)
+        return fail(DCP_ERR_MISALIGNED, "%s: out_stride_n %lld elements is not a multiple of 16 bytes", fn,
+                    (long long)out_stride_n);
+    if (B == 0) return ok();
+    if (!outputs || !lses || !result) return fail(DCP_ERR_INVALID_ARG, "%s: null buffer pointer", fn);
+    if (return_lse && !global_lse) return fail(DCP_ERR_INVALID_ARG, "%s: return_lse set but global_lse is null", fn);
+    if (!aligned(outputs, 16) || !aligned(result, 16))
+        return fail(DCP_ERR_MISALIGNED, "%s: outputs and result must be 16-byte aligned", fn);
+    if (!aligned(lses, 4) || (return_lse && !aligned(global_lse, 4)))
+        return fail(DCP_ERR_MISALIGNED, "%s: lses and global_lse must be 4-byte aligned", fn);
+
+    dcp::CombineArgs a{};
+    a.src = static_cast<const uint32_t *>(outputs);
+    a.lses = lses;
+    a.result = static_cast<uint32_t *>(result);
+    a.glse = global_lse;
+    a.units = B * H;
+    a.shard_stride_w = out_stride_n * es / 4;
+    a.lse_stride_n = lse_stride_n;
+    a.data_w = (int32_t)(D * es / 4);
+    a.row_pitch_w = a.data_w;
+    a.chunks = a.data_w / 4;
+    a.N = N;
+    a.base_e = is_lse_base_on_e ? 1 : 0;
+    a.return_lse = return_lse ? 1 : 0;
+    return dispatch_dtype<false>(dtype, a, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int32_t dcp_unpack_combine(const void *recv_buf, void *result, float *global_lse, int32_t N, int64_t B, int64_t Hr,
+                           int64_t D, int64_t stride_n, int32_t dtype, int32_t is_lse_base_on_e, int32_t return_lse,
+                           void *cuda_stream) {
+    const char *fn = "dcp_unpack_combine";
+    int32_t st = check_common(fn, dtype, N, B, Hr, D);
+    if (st != DCP_OK) return st;
+    const int es = elem_size(dtype);
+    const int64_t W = D + 4 / es;
+    if (stride_n < B * Hr * W)
+        return fail(DCP_ERR_INVALID_ARG, "%s: stride_n %lld < B*Hr*(D+P) = %lld", fn, (long long)stride_n,
+                    (long long)(B * Hr * W));
+    if ((stride_n * es) % 4 != 0)
+        return fail(DCP_ERR_MISALIGNED, "%s: stride_n %lld elements is not a multiple of 4 bytes", fn,
+                    (long long)stride_n);
+    if (B == 0) return ok();
+    if (!recv_buf || !result) return fail(DCP_ERR_INVALID_ARG, "%s: null buffer pointer", fn);
+    if (return_lse && !global_lse) return fail(DCP_ERR_INVALID_ARG, "%s: return_lse set but global_lse is null", fn);
+    if (!aligned(recv_buf, 16) || !aligned(result, 16))
+        return fail(DCP_ERR_MISALIGNED, "%s: recv_buf and result must be 16-byte aligned", fn);
+    if (return_lse && !aligned(global_lse, 4))
+        return fail(DCP_ERR_MISALIGNED, "%s: global_lse must be 4-byte aligned", fn);
+
+    dcp::CombineArgs a{};
+    a.src = static_cast<const uint32_t *>(recv_buf);
+    a.lses = nullptr;
+    a.result = static_cast<uint32_t *>(result);
+    a.glse = global_lse;
+    a.units = B * Hr;
+    a.shard_stride_w = stride_n * es / 4;
+    a.lse_stride_n = 0;
+    a.data_w = (int32_t)(D * es / 4);
+    a.row_pitch_w = a.data_w + 1;
+    a.chunks = a.data_w;
+    a.N = N;
+    a.base_e = is_lse_base_on_e ? 1 : 0;
+    a.return_lse = return_lse ? 1 : 0;
+    return dispatch_dtype<true>(dtype, a, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_buf, int64_t B, int64_t H, int64_t D,
+                 int32_t world_size, int32_t dtype, int64_t out_stride_b, int64_t out_stride_h, int64_t lse_stride_b,
+                 void *cuda_stream) {
+    const char *fn = "dcp_pack";
+    int32_t st = check_common(fn, dtype, world_size, B, H, D);
+    if (st != DCP_OK) return st;
+    if (H % world_size != 0)
+        return fail(DCP_ERR_SHAPE, "%s: H=%lld heads do not split evenly over %d ranks", fn, (long long)H,
+                    (int)world_size);
+    const int es = elem_size(dtype);
+    if (out_stride_b < 1 || out_stride_h < 1)
+        return fail(DCP_ERR_INVALID_ARG, "%s: output strides must be >= 1", fn);
+    if ((out_stride_b * es) % 16 != 0 || (out_stride_h * es) % 16 != 0)
+        return fail(DCP_ERR_MISALIGNED, "%s: output strides (%lld, %lld) are not multiples of 16 bytes", fn,
+                    (long long)out_stride_b, (long long)out_stride_h);
+    if (lse_stride_b < H)
+        return fail(DCP_ERR_INVALID_ARG, "%s: lse_stride_b %lld < H = %lld", fn, (long long)lse_stride_b,
+                    (long long)H);
+    if (B == 0) return ok();
+    if (!cp_attn_out || !cp_attn_lse || !send_buf) return fail(DCP_ERR_INVALID_ARG, "%s: null buffer pointer", fn);
+    if (!aligned(cp_attn_out, 16) || !aligned(send_buf, 16))
+        return fail(DCP_ERR_MISALIGNED, "%s: cp_attn_out and send_buf must be 16-byte aligned", fn);
+    if (!aligned(cp_attn_lse, 4)) return fail(DCP_ERR_MISALIGNED, "%s: cp_attn_lse must be 4-byte aligned", fn);
+
+    dcp::PackArgs a{};
+    a.src = static_cast<const uint32_t *>(cp_attn_out);
+    a.lse = reinterpret_cast<const uint32_t *>(cp_attn_lse);
+    a.dst = static_cast<uint32_t *>(send_buf);
+    a.B = B;
+    a.Hr = H / world_size;
+    a.rows = (int64_t)world_size * B * a.Hr;
+    a.src_stride_b_w = out_stride_b * es / 4;
+    a.src_stride_h_w = out_stride_h * es / 4;
+    a.lse_stride_b = lse_stride_b;
+    a.data_w = (int32_t)(D * es / 4);
+    a.chunks = a.data_w / 4;
+    a.chunks_magic = ((uint64_t(1) << 32) + (uint64_t)a.chunks - 1) / (uint64_t)a.chunks;
+    a.row_pitch_w = a.data_w + 1;
+    // a tile of about 16 KiB of packed rows (at most one row per thread)
+    int tile_rows = 4096 / a.row_pitch_w;
+    if (tile_rows < 1) tile_rows = 1;
+    if (tile_rows > dcp::kPackThreads) tile_rows = dcp::kPackThreads;
+    a.tile_rows = tile_rows;
+    const size_t smem = (size_t)((3 + (int64_t)tile_rows * a.row_pitch_w + 3) / 4) * 16;
+
+    static const int per_sm = resident_ctas(dcp::pack_kernel, dcp::kPackThreads, 4 * 4096 + 64);
+    const int64_t tiles = (a.rows + tile_rows - 1) / tile_rows;
+    const int64_t cap = (int64_t)sm_count() * per_sm;
+    const int grid = (int)(tiles < cap ? tiles : cap);
+    dcp::pack_kernel<<<grid, dcp::kPackThreads, smem, static_cast<cudaStream_t>(cuda_stream)>>>(a);
+    return launch_status(fn);
+}
+
+}  // extern "C"

@@ -1,0 +1,162 @@
+/*
+ * dcp_combine.h -- C ABI of libdcpcombine.so: the decode-context-parallel (DCP)
+ * LSE-weighted combine of partial attention outputs on NVIDIA B200 (sm_100a).
+ *
+ * Decode context parallelism shards the KV cache of each request over N ranks.
+ * Each shard attends to its part of the context and returns a partial output
+ * [B, H, D] with its log-sum-exp (LSE) [B, H]; the exact attention result is
+ * the LSE-weighted combine of the N partials.  This library runs the three
+ * device steps of that combine, all inside one GPU's memory:
+ *
+ *   dcp_pack            partial output + fp32 LSE -> one packed send buffer
+ *   dcp_lse_combine     combine of separate output / LSE receive buffers
+ *   dcp_unpack_combine  combine read straight out of the packed buffer
+ *
+ * Defining passages (web pages, by title and section):
+ *   [COMBINE] vLLM API docs, vllm.v1.attention.ops.dcp_alltoall,
+ *             _lse_weighted_combine: the combine rules.
+ *   [A2A]     same page, dcp_a2a_lse_reduce: the packed buffer
+ *             [N, B, H/N, D + lse_pack_dim] in the output dtype, the head
+ *             scatter (rank r receives heads [r*H/N, (r+1)*H/N)), and the
+ *             unpack+combine that follows the All-to-All.
+ *   [DIRECT]  vLLM API docs, vllm.v1.attention.ops.dcp, DirectDCPA2AWorkspace:
+ *             split receive buffers received_output [N, T_max, H/N, D] and
+ *             received_lse [N, T_max, H/N] (fp32), i.e. a shard stride that
+ *             may exceed B*H*D.
+ *
+ * The combine, per token b and head h, over shards n = 0..N-1 ([COMBINE]):
+ *   l_n <- -inf if l_n is NaN or +-inf
+ *   m    = max_n l_n, and m <- 0 if m == -inf
+ *   w_n  = exp(l_n - m) (base e) or 2^(l_n - m) (base 2); NaN -> 0
+ *   S    = sum_n w_n;  w_n <- w_n / max(S, 1e-10)
+ *   out[b,h,:]    = sum_n w_n * o_n[b,h,:]   (fp32 accumulation, one rounding)
+ *   global_lse[b,h] = ln(S) + m   (log2(S) + m in base 2; S unclamped, so an
+ *                                  all-empty row gives -inf)
+ *
+ * Conventions shared by every entry point:
+ *   - All buffer pointers are DEVICE pointers on the device that is current on
+ *     the calling thread; the caller owns every buffer.  The library allocates
+ *     nothing and keeps no state besides a per-thread error message.
+ *   - Calls are asynchronous on `cuda_stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and never synchronise.  Inputs must stay valid
+ *     and outputs untouched until the stream reaches the call.
+ *   - Outputs must not overlap inputs.
+ *   - Sizes and strides are in ELEMENTS of the named array's type.
+ *   - Every argument is validated on the host before any launch; a non-zero
+ *     dcp_status is returned and nothing is launched.  dcp_last_error() then
+ *     describes the problem.  A failed launch returns DCP_ERR_CUDA.
+ *   - B == 0 is a valid no-op.
+ *   - Thread-safe: no global mutable state (the error text is thread-local).
+ */
+#ifndef DCP_COMBINE_H
+#define DCP_COMBINE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of the attention outputs and of the packed buffer.  LSEs are
+ * always fp32 ([A2A]: "cp_attn_lse: [B, H] log-sum-exp values (fp32)"). */
+typedef enum {
+    DCP_BF16 = 0,
+    DCP_FP16 = 1,
+    DCP_FP32 = 2
+} dcp_dtype;
+
+typedef enum {
+    DCP_OK = 0,
+    DCP_ERR_INVALID_ARG = 1,       /* null pointer, count out of range, bad stride */
+    DCP_ERR_UNSUPPORTED_DTYPE = 2, /* dtype not one of dcp_dtype */
+    DCP_ERR_MISALIGNED = 3,        /* pointer / row / stride alignment not met */
+    DCP_ERR_SHAPE = 4,             /* H not divisible by world_size */
+    DCP_ERR_CUDA = 5               /* the kernel launch failed */
+} dcp_status;
+
+/* Largest number of shards (DCP ranks) one call combines. */
+#define DCP_MAX_SHARDS 64
+
+/*
+ * Number of output-dtype slots that carry one fp32 LSE in a packed row
+ * ([A2A], _dcp_a2a_lse_pack_dim): 4 bytes / element size, i.e. 2 for bf16
+ * and fp16, 1 for fp32.  Returns -1 for an unknown dtype.
+ */
+int32_t dcp_lse_pack_dim(int32_t dtype);
+
+/*
+ * Pack step of [A2A] dcp_a2a_lse_reduce.
+ *
+ * cp_attn_out  [B, H, D] of `dtype`; element (b, h, d) at
+ *              b*out_stride_b + h*out_stride_h + d.
+ * cp_attn_lse  [B, H] fp32; element (b, h) at b*lse_stride_b + h.
+ * send_buf     [world_size, B, H/world_size, D + P] of `dtype`, contiguous,
+ *              P = dcp_lse_pack_dim(dtype).  Row (r, b, h) receives
+ *              cp_attn_out[b, r*H/world_size + h, 0:D] unchanged, then the 4
+ *              bytes of cp_attn_lse[b, r*H/world_size + h] in memory order
+ *              (slot D = low half-word for 16-bit dtypes).  Bit-exact: no
+ *              rounding, NaN payloads preserved.
+ *
+ * Requirements: world_size in [1, DCP_MAX_SHARDS]; H % world_size == 0
+ * (else DCP_ERR_SHAPE); B >= 0; H, D >= 1; D*elemsize a multiple of 16
+ * (D % 8 == 0 for 16-bit types, D % 4 == 0 for fp32); cp_attn_out and
+ * send_buf 16-byte aligned, out_stride_b / out_stride_h multiples of
+ * 16/elemsize and >= 1 (else DCP_ERR_MISALIGNED / DCP_ERR_INVALID_ARG);
+ * cp_attn_lse 4-byte aligned, lse_stride_b >= H.
+ */
+int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_buf,
+                 int64_t B, int64_t H, int64_t D, int32_t world_size, int32_t dtype,
+                 int64_t out_stride_b, int64_t out_stride_h, int64_t lse_stride_b,
+                 void *cuda_stream);
+
+/*
+ * Combine of split receive buffers ([COMBINE] on the [DIRECT] layout).
+ *
+ * outputs     [N, B, H, D] of `dtype`; element (n, b, h, d) at
+ *             n*out_stride_n + (b*H + h)*D + d, out_stride_n >= B*H*D.
+ * lses        [N, B, H] fp32; element (n, b, h) at n*lse_stride_n + b*H + h,
+ *             lse_stride_n >= B*H.
+ * result      [B, H, D] of `dtype`, contiguous.
+ * global_lse  [B, H] fp32, contiguous; written only when return_lse != 0
+ *             (may be NULL otherwise).
+ * is_lse_base_on_e  nonzero: LSEs are natural logs; zero: base-2 logs.
+ *
+ * Requirements: N in [1, DCP_MAX_SHARDS]; B >= 0; H, D >= 1; D*elemsize a
+ * multiple of 16; outputs and result 16-byte aligned; out_stride_n a
+ * multiple of 16/elemsize; lses and global_lse 4-byte aligned.
+ */
+int32_t dcp_lse_combine(const void *outputs, const float *lses, void *result, float *global_lse,
+                        int32_t N, int64_t B, int64_t H, int64_t D,
+                        int64_t out_stride_n, int64_t lse_stride_n, int32_t dtype,
+                        int32_t is_lse_base_on_e, int32_t return_lse, void *cuda_stream);
+
+/*
+ * Fused unpack + combine over the packed receive buffer ([A2A], the step
+ * after the All-to-All): one pass over the buffer, the LSE read out of each
+ * row's last P slots.
+ *
+ * recv_buf    [N, B, Hr, D + P] of `dtype`; row (n, b, h) starts at element
+ *             n*stride_n + (b*Hr + h)*(D + P); stride_n >= B*Hr*(D + P).
+ * result      [B, Hr, D] of `dtype`, contiguous.
+ * global_lse  [B, Hr] fp32, contiguous; written only when return_lse != 0.
+ *
+ * Requirements: N in [1, DCP_MAX_SHARDS]; B >= 0; Hr, D >= 1; D*elemsize a
+ * multiple of 16; recv_buf and result 16-byte aligned; stride_n*elemsize a
+ * multiple of 4; global_lse 4-byte aligned.
+ */
+int32_t dcp_unpack_combine(const void *recv_buf, void *result, float *global_lse,
+                           int32_t N, int64_t B, int64_t Hr, int64_t D, int64_t stride_n,
+                           int32_t dtype, int32_t is_lse_base_on_e, int32_t return_lse,
+                           void *cuda_stream);
+
+/* Text of the last non-OK status returned on the calling thread ("" if none). */
+const char *dcp_last_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t dcp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCP_COMBINE_H */

@@ -1,0 +1,90 @@
+"""Host-side logic of bench.py on the CPU: the reference (CPU oracle) arm's JSON line, and the
+multi-rank plumbing -- per-rank batches and max-over-ranks timing -- with world_size 2 over gloo."""
+from __future__ import annotations
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _run_bench(args, env_extra=None):
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True, text=True,
+                          env=env, timeout=600, cwd=ROOT)
+
+
+def test_reference_arm_prints_one_line():
+    r = _run_bench(["--impl", "reference", "--steps", "2", "--warmup", "1", "--workload", "sweep_N2_B512_D128"])
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["higher_is_better"] is True
+    assert line["config"]["workload"] == "sweep_N2_B512_D128"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_silently():
+    r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "0"], {"RANK": "1", "WORLD_SIZE": "2"})
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
+
+
+def test_rank_seeds_are_distinct():
+    seeds = {bench.rank_seed(100, r) for r in range(8)}
+    assert len(seeds) == 8
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # per-rank inputs differ (weak scaling: each rank its own batch of the same shape)
+        from decode_context_attention_dcp_b200 import workloads as wl
+        w = wl.TINY.with_(seed=bench.rank_seed(wl.TINY.seed, rank))
+        cp_out, _ = wl.pack_inputs(w)
+        gathered = [torch.zeros_like(cp_out.float()) for _ in range(world)]
+        dist.all_gather(gathered, cp_out.float())
+        distinct = not torch.equal(gathered[0], gathered[1])
+        bench.barrier()
+        m = bench.max_over_ranks(float(rank + 1) * 1.5)
+        out[rank] = (m, distinct, tuple(cp_out.shape))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+        assert p.exitcode == 0
+    assert out[0][0] == 3.0 and out[1][0] == 3.0
+    assert out[0][1] and out[1][1]
+    assert out[0][2] == out[1][2] == (4, 16, 128)

@@ -1,0 +1,345 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on the seeded DCP workloads.
+
+Element by element wherever the oracle finishes in seconds; at the largest sizes on sampled
+(token, head) rows plus properties that hold everywhere.  Pack is compared bit for bit.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import decode_context_attention_dcp_b200 as dcp
+import oracle as orc
+import oracle_pins
+from decode_context_attention_dcp_b200 import workloads as wl
+from gpu_util import (ORACLE_CODE, Guarded, as_f64, assert_lse_close, assert_out_close, packed_from_split, raw,
+                      sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def o() -> orc.Oracle:
+    return orc.load()
+
+
+def gpu_combine(outputs, lses, w: wl.CombineWorkload, return_lse=None):
+    ret = w.return_lse if return_lse is None else return_lse
+    return dcp.lse_weighted_combine(outputs.cuda(), lses.cuda(), return_lse=ret,
+                                    is_lse_base_on_e=w.is_lse_base_on_e)
+
+
+def gpu_unpack(recv, w: wl.CombineWorkload, return_lse=None):
+    ret = w.return_lse if return_lse is None else return_lse
+    return dcp.unpack_combine(recv.cuda(), return_lse=ret, is_lse_base_on_e=w.is_lse_base_on_e)
+
+
+def check_split(o, w, outputs, lses, ret):
+    code = ORACLE_CODE[outputs.dtype]
+    got = gpu_combine(outputs, lses, w, ret)
+    ref = o.lse_combine(raw(outputs), code, raw(lses), return_lse=ret, is_lse_base_on_e=w.is_lse_base_on_e)
+    if ret:
+        assert_out_close(got[0], ref[0], f"{w.name} combine")
+        assert_lse_close(got[1], ref[1], f"{w.name} combine lse")
+    else:
+        assert_out_close(got, ref, f"{w.name} combine")
+    return got, ref
+
+
+def check_packed(o, w, recv, ret):
+    code = ORACLE_CODE[recv.dtype]
+    got = gpu_unpack(recv, w, ret)
+    ref = o.unpack_combine(raw(recv), code, w.D, return_lse=ret, is_lse_base_on_e=w.is_lse_base_on_e)
+    if ret:
+        assert_out_close(got[0], ref[0], f"{w.name} unpack_combine")
+        assert_lse_close(got[1], ref[1], f"{w.name} unpack_combine lse")
+    else:
+        assert_out_close(got, ref, f"{w.name} unpack_combine")
+    return got, ref
+
+
+# ---- the four named workloads, element by element ------------------------------------------
+def test_tiny(o):
+    w = wl.TINY
+    outputs, lses = wl.split_inputs(w)
+    check_split(o, w, outputs, lses, True)
+    check_packed(o, w, packed_from_split(outputs, lses), True)
+
+
+@pytest.mark.parametrize("split", ["contiguous", "interleaved"])
+@pytest.mark.parametrize("base_e", [True, False])
+def test_tiny_bruteforce_attention(o, split, base_e):
+    """K/V of length 64 split over 2 shards: per-shard attention + LSE (fp64, rounded to bf16 /
+    fp32 as a shard would emit them), combined on the GPU, equals full attention."""
+    case = wl.AttentionCase()
+    q, k, v = wl.attention_inputs(case)
+    scale = 1.0 / math.sqrt(case.D)
+    shards = oracle_pins.shard_positions(case.L, case.N, split)
+    outs = np.zeros((case.N, case.B, case.H, case.D))
+    lses = np.zeros((case.N, case.B, case.H))
+    full_o = np.zeros((case.B, case.H, case.D))
+    full_l = np.zeros((case.B, case.H))
+    for b in range(case.B):
+        qb, kb, vb = raw(q[b]), raw(k[b]), raw(v[b])
+        full_o[b], full_l[b] = o.attention(qb, kb, vb, orc.BF16, list(range(case.L)), scale, base_e)
+        for r, pos in enumerate(shards):
+            outs[r, b], lses[r, b] = o.attention(qb, kb, vb, orc.BF16, pos, scale, base_e)
+    shard_out = torch.from_numpy(outs).to(torch.bfloat16)
+    shard_lse = torch.from_numpy(lses).to(torch.float32)
+    y, g = dcp.lse_weighted_combine(shard_out.cuda(), shard_lse.cuda(), return_lse=True, is_lse_base_on_e=base_e)
+    assert_out_close(y, full_o, "combine vs full attention")
+    assert_lse_close(g, full_l, "global lse vs full attention")
+    # the same through the packed layout
+    y2, g2 = dcp.unpack_combine(packed_from_split(shard_out, shard_lse).cuda(), return_lse=True,
+                                is_lse_base_on_e=base_e)
+    assert_out_close(y2, full_o, "unpack_combine vs full attention")
+    assert_lse_close(g2, full_l, "unpack_combine lse vs full attention")
+
+
+@pytest.mark.parametrize("ret", [False, True])
+def test_gqa_packed(o, ret):
+    w = wl.GQA
+    outputs, lses = wl.split_inputs(w)
+    assert torch.isnan(lses).any() and torch.isinf(lses).any()
+    check_packed(o, w, packed_from_split(outputs, lses), ret)
+    check_split(o, w, outputs, lses, ret)
+
+
+def test_mla(o):
+    w = wl.MLA
+    outputs, lses = wl.split_inputs(w)
+    (y, g), _ = check_split(o, w, outputs, lses, True)
+    empty = torch.arange(w.B) % w.empty_every == 0
+    assert bool((y[empty.cuda()] == 0).all())
+    assert bool((g[empty.cuda()] == -math.inf).all())
+    assert bool(torch.isfinite(g[~empty.cuda()]).all())
+
+
+def test_mla_through_pack(o):
+    """MLA shards laid out as one rank's cp_attn_out [B, N*Hr, D]: pack (bit-exact), then unpack+combine
+    over the packed buffer with every shard taken from it."""
+    w = wl.MLA
+    outputs, lses = wl.split_inputs(w)
+    cp_out = outputs.permute(1, 0, 2, 3).reshape(w.B, w.H, w.D).contiguous()
+    cp_lse = lses.permute(1, 0, 2).reshape(w.B, w.H).contiguous()
+    send = dcp.pack(cp_out.cuda(), cp_lse.cuda(), w.N)
+    ref_send = o.pack(raw(cp_out), raw(cp_lse), w.N, orc.BF16)
+    assert np.array_equal(raw(send.cpu()), ref_send), "pack is not bit-exact"
+    y, g = dcp.unpack_combine(send, return_lse=True, is_lse_base_on_e=False)
+    ry, rg = o.unpack_combine(ref_send, orc.BF16, w.D, return_lse=True, is_lse_base_on_e=False)
+    assert_out_close(y, ry, "mla unpack_combine")
+    assert_lse_close(g, rg, "mla unpack_combine lse")
+
+
+def test_roundtrip_fp16(o):
+    w = wl.ROUNDTRIP
+    cp_out, cp_lse = wl.pack_inputs(w)
+    assert cp_out.shape == (2048, 64, 128) and cp_out.dtype == torch.float16
+    send = dcp.pack(cp_out.cuda(), cp_lse.cuda(), w.N)
+    assert send.shape == (8, 2048, 8, 130)
+    ref_send = o.pack(raw(cp_out), raw(cp_lse), w.N, orc.FP16)
+    assert np.array_equal(raw(send.cpu()), ref_send), "pack is not bit-exact"
+    y = dcp.unpack_combine(send)
+    ry = o.unpack_combine(ref_send, orc.FP16, w.D)
+    assert_out_close(y, ry, "roundtrip unpack_combine")
+
+
+# ---- the bandwidth sweep -----------------------------------------------------------------
+SWEEP = wl.sweep()
+SWEEP_SMALL = [p for p in SWEEP if p.B == 512]
+SWEEP_LARGE = [p for p in SWEEP if p.B == 16384]
+
+
+@pytest.mark.parametrize("w", SWEEP_SMALL, ids=lambda p: p.name)
+def test_sweep_full_elementwise(o, w):
+    outputs, lses = wl.split_inputs(w)
+    check_split(o, w, outputs, lses, False)
+    check_packed(o, w, packed_from_split(outputs, lses), False)
+
+
+@pytest.mark.parametrize("w", SWEEP_LARGE, ids=lambda p: p.name)
+def test_sweep_full_size_sampled(o, w):
+    """Full-size inputs; both entry points checked on sampled rows against the oracle, and
+    everywhere for finiteness (the inputs are finite and the LSEs never all -inf together)."""
+    outputs, lses = wl.split_inputs(w)
+    d_out, d_lse = outputs.cuda(), lses.cuda()
+    y = dcp.lse_weighted_combine(d_out, d_lse)
+    recv = torch.cat([d_out, d_lse.unsqueeze(-1).view(d_out.dtype)], dim=-1)
+    del d_out
+    y2 = dcp.unpack_combine(recv)
+    del recv
+    assert bool(torch.isfinite(y).all()) and bool(torch.isfinite(y2).all())
+    rows = sample_rows(w.B, w.Hr, 48, w.seed)
+    ref, _ = o.lse_combine_rows(raw(outputs), orc.BF16, raw(lses), rows)
+    bi = torch.tensor([r[0] for r in rows])
+    hi = torch.tensor([r[1] for r in rows])
+    assert_out_close(y.cpu()[bi, hi], ref, f"{w.name} combine (sampled)")
+    assert_out_close(y2.cpu()[bi, hi], ref, f"{w.name} unpack_combine (sampled)")
+
+
+def test_bench_step_full_size(o):
+    """The bench's step at full size (largest sweep point): pack of cp_attn_out [B, N*Hr, D]
+    compared bit for bit everywhere, then unpack+combine of the send buffer on sampled rows."""
+    w = wl.by_name("sweep_N16_B16384_D512")
+    cp_out, cp_lse = wl.pack_inputs(w)
+    send = dcp.pack(cp_out.cuda(), cp_lse.cuda(), w.N)
+    ref_send = o.pack(raw(cp_out), raw(cp_lse), w.N, orc.BF16)
+    del cp_out
+    got_send = raw(send.cpu())
+    assert np.array_equal(got_send, ref_send), "pack is not bit-exact"
+    del got_send
+    y = dcp.unpack_combine(send, is_lse_base_on_e=w.is_lse_base_on_e)
+    rows = sample_rows(w.B, w.Hr, 48, 7)
+    ref, _ = o.unpack_combine_rows(ref_send, orc.BF16, w.D, rows)
+    bi = torch.tensor([r[0] for r in rows])
+    hi = torch.tensor([r[1] for r in rows])
+    assert_out_close(y.cpu()[bi, hi], ref, "bench step unpack_combine (sampled)")
+    assert bool(torch.isfinite(y).all())
+
+
+# ---- shapes, dtypes and edge cases -----------------------------------------------------------
+def _case(N, B, Hr, D, dtype, seed, p_neginf=0.1, p_nan=0.05, base_e=True):
+    w = wl.CombineWorkload(f"edge_N{N}_B{B}_H{Hr}_D{D}_{dtype}", N=N, B=B, Hr=Hr, D=D, dtype=dtype,
+                           p_neginf=p_neginf, p_nan=p_nan, is_lse_base_on_e=base_e, lse_lo=-30.0, lse_hi=30.0,
+                           seed=seed)
+    return w, *wl.split_inputs(w)
+
+
+EDGE = [(N, B, Hr, D, dt)
+        for (N, B, Hr, D) in [(1, 3, 2, 128), (2, 1, 1, 8), (3, 37, 3, 64), (5, 7, 5, 96), (16, 9, 2, 512),
+                              (64, 3, 2, 128), (7, 2, 3, 576), (4, 5, 1, 1024), (2, 129, 4, 16), (33, 4, 3, 256)]
+        for dt in ("bf16", "fp16", "fp32")]
+
+
+@pytest.mark.parametrize("N,B,Hr,D,dtype", EDGE)
+def test_edge_shapes(o, N, B, Hr, D, dtype):
+    if dtype == "fp32" and D % 4:
+        pytest.skip("fp32 rows need D % 4 == 0")
+    seed = (N * 131 + B * 17 + Hr * 7 + D) % 1000
+    for base_e in (True, False):
+        w, outputs, lses = _case(N, B, Hr, D, dtype, seed, base_e=base_e)
+        check_split(o, w, outputs, lses, True)
+        check_packed(o, w, packed_from_split(outputs, lses), True)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16", "fp32"])
+def test_single_shard_is_identity(dtype):
+    w, outputs, lses = _case(1, 6, 4, 128, dtype, 5, p_neginf=0.0, p_nan=0.0)
+    y, g = gpu_combine(outputs, lses, w, True)
+    assert torch.equal(y.cpu().view(torch.int16 if dtype != "fp32" else torch.int32),
+                       outputs[0].view(torch.int16 if dtype != "fp32" else torch.int32))
+    assert torch.equal(g.cpu(), lses[0])
+    y2, g2 = gpu_unpack(packed_from_split(outputs, lses), w, True)
+    assert torch.equal(y2.cpu(), y.cpu()) and torch.equal(g2.cpu(), g.cpu())
+
+
+def test_special_lses(o):
+    """NaN, +inf and -inf LSEs, all-empty rows and single-finite-shard rows."""
+    w, outputs, lses = _case(4, 8, 2, 128, "bf16", 3, p_neginf=0.0, p_nan=0.0)
+    lses[:, 0, :] = float("-inf")
+    lses[:, 1, :] = torch.tensor([float("nan"), float("inf"), float("-inf"), float("nan")]).unsqueeze(-1)
+    lses[:, 2, 0] = torch.tensor([float("nan"), 3.0, float("inf"), float("-inf")])
+    lses[:, 3, 1] = float("inf")
+    lses[2, 4, :] = float("inf")
+    (y, g), _ = check_split(o, w, outputs, lses, True)
+    check_packed(o, w, packed_from_split(outputs, lses), True)
+    assert bool((y.cpu()[0:2] == 0).all()) and bool((g.cpu()[0:2] == -math.inf).all())
+    assert torch.equal(y.cpu()[2, 0], outputs[1, 2, 0])
+    assert float(g.cpu()[2, 0]) == 3.0
+
+
+def test_capacity_strided_shards(o):
+    """Receive buffers with room for T_max > B tokens per shard (the direct-workspace layout)."""
+    N, T_max, B, Hr, D = 4, 50, 37, 3, 128
+    w, outputs, lses = _case(N, T_max, Hr, D, "bf16", 9)
+    d_out, d_lse = outputs.cuda(), lses.cuda()
+    y = torch.empty((B, Hr, D), dtype=torch.bfloat16, device="cuda")
+    g = torch.empty((B, Hr), dtype=torch.float32, device="cuda")
+    dcp.dcp_lse_combine(d_out[:, :B], d_lse[:, :B], y, g, return_lse=True)
+    ry, rg = o.lse_combine(raw(outputs[:, :B]), orc.BF16, raw(lses[:, :B]), return_lse=True)
+    assert_out_close(y, ry, "strided combine")
+    assert_lse_close(g, rg, "strided combine lse")
+    recv = packed_from_split(outputs, lses).cuda()
+    y2 = torch.empty_like(y)
+    g2 = torch.empty_like(g)
+    dcp.dcp_unpack_combine(recv[:, :B], y2, g2, return_lse=True)
+    assert_out_close(y2, ry, "strided unpack_combine")
+    assert_lse_close(g2, rg, "strided unpack_combine lse")
+
+
+def test_outputs_stay_inside_their_buffers(o):
+    w, outputs, lses = _case(3, 33, 3, 96, "bf16", 11)
+    res = Guarded((33, 3, 96), torch.bfloat16)
+    gl = Guarded((33, 3), torch.float32)
+    dcp.dcp_lse_combine(outputs.cuda(), lses.cuda(), res.tensor, gl.tensor, return_lse=True)
+    res.check()
+    gl.check()
+    ry, rg = o.lse_combine(raw(outputs), orc.BF16, raw(lses), return_lse=True)
+    assert_out_close(res.tensor, ry)
+    assert_lse_close(gl.tensor, rg)
+    res2 = Guarded((33, 3, 96), torch.bfloat16)
+    gl2 = Guarded((33, 3), torch.float32)
+    dcp.dcp_unpack_combine(packed_from_split(outputs, lses).cuda(), res2.tensor, gl2.tensor, return_lse=True)
+    res2.check()
+    gl2.check()
+    assert_out_close(res2.tensor, ry)
+    # pack: every packed-row alignment (rows are 4 bytes past a 16-byte boundary each) and ragged tiles
+    for (B, H, D, ws) in [(3, 12, 8, 3), (5, 10, 128, 5), (2, 6, 520, 2), (1, 1, 64, 1), (70, 8, 128, 4)]:
+        out = torch.randn(B, H, D).to(torch.bfloat16)
+        lse = torch.randn(B, H)
+        send = Guarded((ws, B, H // ws, D + 2), torch.bfloat16)
+        dcp.dcp_pack(out.cuda(), lse.cuda(), send.tensor, ws)
+        send.check()
+        assert np.array_equal(raw(send.tensor.cpu()), o.pack(raw(out), raw(lse), ws, orc.BF16)), (B, H, D, ws)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16", "fp32"])
+def test_pack_bit_exact_strided_inputs(o, dtype):
+    dt = wl.torch_dtype(dtype)
+    B, H, D, ws = 7, 12, 64, 4
+    big = torch.randn(B + 1, H + 2, D + 8).to(dt)
+    out = big[1:, 1:H + 1, :D]                 # strides (H+2)*(D+8), D+8, 1
+    lse_big = torch.randn(B, H + 5)
+    lse_big[0, 0] = float("nan")
+    lse_big.view(torch.int32)[0, 1] = 0x7FC01234    # NaN payload must survive
+    lse_big[0, 2] = float("-inf")
+    lse = lse_big[:, :H]
+    send = dcp.pack(out.cuda(), lse.cuda(), ws)
+    ref = o.pack(raw(out.contiguous()), raw(lse.contiguous()), ws, ORACLE_CODE[dt])
+    assert np.array_equal(raw(send.cpu()), ref)
+
+
+def test_empty_batch_is_a_noop():
+    outputs = torch.zeros((2, 0, 4, 128), dtype=torch.bfloat16, device="cuda")
+    lses = torch.zeros((2, 0, 4), device="cuda")
+    y = torch.empty((0, 4, 128), dtype=torch.bfloat16, device="cuda")
+    dcp.dcp_lse_combine(outputs, lses, y)
+    recv = torch.zeros((2, 0, 4, 130), dtype=torch.bfloat16, device="cuda")
+    dcp.dcp_unpack_combine(recv, y)
+    send = torch.empty((2, 0, 2, 130), dtype=torch.bfloat16, device="cuda")
+    dcp.dcp_pack(torch.zeros((0, 4, 128), dtype=torch.bfloat16, device="cuda"),
+                 torch.zeros((0, 4), device="cuda"), send, 2)
+    torch.cuda.synchronize()
+
+
+def test_side_stream(o):
+    w, outputs, lses = _case(8, 64, 4, 128, "bf16", 21)
+    s = torch.cuda.Stream()
+    d_out, d_lse = outputs.cuda(), lses.cuda()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        y = dcp.lse_weighted_combine(d_out, d_lse)
+    s.synchronize()
+    assert_out_close(y, o.lse_combine(raw(outputs), orc.BF16, raw(lses)), "side stream")
+
+
+def test_errors_raise():
+    x = torch.zeros((2, 4, 8, 12), dtype=torch.bfloat16, device="cuda")     # 24-byte rows
+    with pytest.raises(dcp.DCPError) as e:
+        dcp.lse_weighted_combine(x, torch.zeros((2, 4, 8), device="cuda"))
+    assert e.value.status == 3
+    with pytest.raises(ValueError):
+        dcp.pack(torch.zeros((2, 6, 128), dtype=torch.bfloat16, device="cuda"), torch.zeros((2, 6), device="cuda"), 4)
