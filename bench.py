@@ -51,6 +51,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the JSON line: per-kernel GB/s on every workload, as a markdown table")
+    ap.add_argument("--sweep-reps", type=int, default=20)
     return ap.parse_args(argv)
 
 
@@ -250,6 +253,64 @@ def workload_config(w) -> dict:
             "l2": "inputs larger than L2 (no flush between steps)"}
 
 
+# ---- per-kernel sweep ------------------------------------------------------------------------
+def run_sweep(args) -> int:
+    """Median device time of each entry point on every workload (L2 flushed before each timed
+    launch); prints a markdown table."""
+    import torch
+
+    import decode_context_attention_dcp_b200 as dcp
+    from decode_context_attention_dcp_b200 import workloads as wl
+
+    torch.cuda.set_device(0)
+    peak, peak_src = load_peak()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    points = [wl.TINY, wl.GQA, wl.MLA, wl.ROUNDTRIP, *wl.sweep()]
+    print(f"| workload | N | B | Hr | D | dtype | kernel | bytes | us | GB/s | frac of {peak:.0f} ({peak_src}) |")
+    print("|---|---|---|---|---|---|---|---|---|---|---|")
+    for w in points:
+        outputs, lses = wl.split_inputs(w)
+        d_out, d_lse = outputs.cuda(), lses.cuda()
+        del outputs, lses
+        recv = torch.cat([d_out, d_lse.unsqueeze(-1).view(d_out.dtype) if w.elem_bytes == 2 else d_lse.unsqueeze(-1)],
+                         dim=-1)
+        cp_out = d_out.permute(1, 0, 2, 3).reshape(w.B, w.H, w.D).contiguous()
+        cp_lse = d_lse.permute(1, 0, 2).reshape(w.B, w.H).contiguous()
+        res = torch.empty((w.B, w.Hr, w.D), dtype=d_out.dtype, device="cuda")
+        gl = torch.empty((w.B, w.Hr), dtype=torch.float32, device="cuda")
+        send = torch.empty_like(recv)
+        kernels = [
+            ("dcp_lse_combine", w.combine_bytes(),
+             lambda: dcp.dcp_lse_combine(d_out, d_lse, res, gl, is_lse_base_on_e=w.is_lse_base_on_e,
+                                         return_lse=w.return_lse)),
+            ("dcp_unpack_combine", w.combine_bytes(),
+             lambda: dcp.dcp_unpack_combine(recv, res, gl, is_lse_base_on_e=w.is_lse_base_on_e,
+                                            return_lse=w.return_lse)),
+            ("dcp_pack", w.pack_bytes(), lambda: dcp.dcp_pack(cp_out, cp_lse, send, w.N)),
+        ]
+        for name, nbytes, fn in kernels:
+            for _ in range(3):
+                fn()
+            times = []
+            for _ in range(args.sweep_reps):
+                # the flush empties L2 and keeps the GPU busy while the host enqueues the timed
+                # launch, so host-side call overhead never lands between the two events
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                torch.cuda.synchronize()
+                times.append(a.elapsed_time(b))
+            t = statistics.median(times)
+            gbs = nbytes / (t * 1e-3) / 1e9
+            print(f"| {w.name} | {w.N} | {w.B} | {w.Hr} | {w.D} | {w.dtype} | {name} | {nbytes} | {t * 1e3:.1f} | "
+                  f"{gbs:.0f} | {gbs / peak:.3f} |", flush=True)
+        del d_out, d_lse, recv, cp_out, cp_lse, res, gl, send
+        torch.cuda.empty_cache()
+    return 0
+
+
 # ---- our arm ---------------------------------------------------------------------------------
 def run_ours(args) -> int:
     import torch
@@ -298,8 +359,10 @@ def run_ours(args) -> int:
     clocks = None
     sampler = None
     if not args.no_clocks:
-        uuid = getattr(torch.cuda.get_device_properties(device), "uuid", None)
-        sampler = ClockSampler(f"GPU-{uuid}" if uuid else None)
+        props = torch.cuda.get_device_properties(device)
+        pci = (f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+               if hasattr(props, "pci_bus_id") else None)
+        sampler = ClockSampler(pci)
         sampler.start()
     with torch.cuda.stream(stream):
         for _ in range(W):
@@ -412,6 +475,8 @@ def main(argv=None) -> int:
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_ours(args)
 
 

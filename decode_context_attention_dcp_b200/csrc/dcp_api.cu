@@ -69,6 +69,32 @@ int resident_ctas(K kernel, int threads, size_t smem) {
     return n;
 }
 
+// The pack kernel's dynamic shared memory can exceed the default 48 KiB: opt in
+// once per device, for the largest stage any accepted row width needs.
+bool pack_smem_reserved() {
+    static std::atomic<int> done[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (dev < 64 && done[dev].load(std::memory_order_acquire)) return true;
+    const int max_stage_w = (int)(((kMaxD + 1 + 3) & ~int64_t(3)) + 4);  // one fp32 row of kMaxD words
+    const size_t bytes = (size_t)dcp::kPackStages * max_stage_w * 4;
+    if (cudaFuncSetAttribute(dcp::pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return false;
+    if (dev < 64) done[dev].store(1, std::memory_order_release);
+    return true;
+}
+
+// Resident pack CTAs per SM for a given dynamic shared-memory size (one cached entry).
+int pack_resident_ctas(size_t smem) {
+    static std::atomic<uint64_t> cache{0};  // (smem << 16) | ctas
+    const uint64_t c = cache.load(std::memory_order_relaxed);
+    if (c && (c >> 16) == smem) return (int)(c & 0xffff);
+    const int n = resident_ctas(dcp::pack_kernel, dcp::kPackThreads, smem);
+    cache.store(((uint64_t)smem << 16) | (uint64_t)n, std::memory_order_relaxed);
+    return n;
+}
+
 int32_t launch_status(const char *what) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DCP_ERR_CUDA, "%s: kernel launch failed: %s", what, cudaGetErrorString(e));
@@ -77,49 +103,95 @@ int32_t launch_status(const char *what) {
 
 // ---------------------------------------------------------------------------
 // combine dispatch
-template <class T, int VW, int G, int CPL, int NB, bool PACKED>
+
+// Per kernel instance: dynamic shared-memory opt-in (once per device) and the
+// resident-CTA count for the last shared-memory size seen.
+struct InstanceCache {
+    std::atomic<int> opted[64];
+    std::atomic<uint64_t> occupancy{0};  // (smem << 16) | ctas
+};
+
+template <class K>
+bool reserve_smem(K kernel, InstanceCache &ic, size_t max_bytes) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (dev < 64 && ic.opted[dev].load(std::memory_order_acquire)) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_bytes) != cudaSuccess)
+        return false;
+    if (dev < 64) ic.opted[dev].store(1, std::memory_order_release);
+    return true;
+}
+
+template <class K>
+int cached_resident_ctas(K kernel, InstanceCache &ic, int threads, size_t smem) {
+    const uint64_t c = ic.occupancy.load(std::memory_order_relaxed);
+    if (c && (c >> 16) == smem) return (int)(c & 0xffff);
+    const int n = resident_ctas(kernel, threads, smem);
+    ic.occupancy.store(((uint64_t)smem << 16) | (uint64_t)n, std::memory_order_relaxed);
+    return n;
+}
+
+template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS>
 int32_t launch_combine(const dcp::CombineArgs &a, cudaStream_t stream) {
-    auto kernel = dcp::combine_kernel<T, VW, G, CPL, NB, PACKED>;
-    static const int per_sm = resident_ctas(kernel, dcp::kCombineThreads, 0);
+    const char *fn = PACKED ? "dcp_unpack_combine" : "dcp_lse_combine";
+    auto kernel = dcp::combine_kernel<T, G, CPL, NB, PACKED, MIN_CTAS>;
+    static InstanceCache ic;
     constexpr int kUnitsPerWarp = 32 / G;
     constexpr int kWarps = dcp::kCombineThreads / 32;
+    const size_t smem = dcp::combine_smem_bytes(kUnitsPerWarp, a.N, PACKED);
+    if (!reserve_smem(kernel, ic, dcp::combine_smem_bytes(kUnitsPerWarp, DCP_MAX_SHARDS, PACKED)))
+        return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
+    const int per_sm = cached_resident_ctas(kernel, ic, dcp::kCombineThreads, smem);
     const int64_t tasks = (a.units + kUnitsPerWarp - 1) / kUnitsPerWarp;
     const int64_t want = (tasks + kWarps - 1) / kWarps;
     const int64_t cap = (int64_t)sm_count() * per_sm;
     const int grid = (int)(want < cap ? want : cap);
-    kernel<<<grid, dcp::kCombineThreads, 0, stream>>>(a);
-    return launch_status(PACKED ? "dcp_unpack_combine" : "dcp_lse_combine");
+    kernel<<<grid, dcp::kCombineThreads, smem, stream>>>(a);
+    return launch_status(fn);
 }
 
-// Lanes per row G: the smallest power of two >= the row's chunk count (at
-// least 4, at most 32).  Chunk slots per lane: ceil(chunks / G), CPL of them
-// per pass, with the loads of NB shards issued before their FMAs, so each lane
-// keeps NB * CPL * VW words in flight (32 for 16-byte chunks, 16 for words).
-template <class T, int VW, bool PACKED>
+// Occupancy: the kernel keeps NB * CPL 16-byte loads in flight per lane, so the
+// bytes in flight per SM are set by how many warps fit.  Capping registers so
+// that 3 CTAs fit (2 for the four-slot shapes, which spill otherwise) measured
+// best on B200 for every shape.
+template <class T, int G, bool PACKED>
+int32_t launch_cpl(dcp::CombineArgs a, int cpl, cudaStream_t stream) {
+    switch (cpl) {
+        case 1: return launch_combine<T, G, 1, 8, PACKED, 3>(a, stream);
+        case 2: return launch_combine<T, G, 2, 4, PACKED, 3>(a, stream);
+        default: return launch_combine<T, G, 4, 2, PACKED, 2>(a, stream);
+    }
+}
+
+// Shape of the work per lane.  Each lane should keep about eight 16-byte loads
+// in flight: chunk slots per lane (CPL) times shards per batch (NB = 8 / CPL),
+// so fewer shards ask for more chunks per lane, i.e. fewer lanes per row (G).
+// The packed layout never goes below two slots per lane: its per-shard
+// realignment favours fewer, longer lane groups.
+template <class T, bool PACKED>
 int32_t dispatch_combine(dcp::CombineArgs a, cudaStream_t stream) {
-    const int ch = a.chunks;
-    constexpr int kSmallNB = VW == 4 ? 8 : 16;
-    if (ch <= 4) { a.slots = 1; return launch_combine<T, VW, 4, 1, kSmallNB, PACKED>(a, stream); }
-    if (ch <= 8) { a.slots = 1; return launch_combine<T, VW, 8, 1, kSmallNB, PACKED>(a, stream); }
-    if (ch <= 16) { a.slots = 1; return launch_combine<T, VW, 16, 1, kSmallNB, PACKED>(a, stream); }
-    a.slots = (ch + 31) / 32;
-    if (a.slots == 1) return launch_combine<T, VW, 32, 1, kSmallNB, PACKED>(a, stream);
-    if constexpr (VW == 4) {
-        return launch_combine<T, VW, 32, 2, 4, PACKED>(a, stream);
-    } else {
-        if (a.slots == 2) return launch_combine<T, VW, 32, 2, 8, PACKED>(a, stream);
-        if (a.slots <= 4) return launch_combine<T, VW, 32, 4, 4, PACKED>(a, stream);
-        return launch_combine<T, VW, 32, 8, 2, PACKED>(a, stream);
+    const int chunks = a.chunks;
+    int cpl_target = a.N >= 8 ? 1 : a.N >= 4 ? 2 : 4;
+    if (PACKED && cpl_target < 2) cpl_target = 2;
+    const int per_lane = (chunks + cpl_target - 1) / cpl_target;
+    int G = 4;
+    while (G < per_lane && G < 32) G *= 2;
+    a.slots = (chunks + G - 1) / G;
+    const int cpl = a.slots >= 3 ? 4 : a.slots;
+    switch (G) {
+        case 4: return launch_cpl<T, 4, PACKED>(a, cpl, stream);
+        case 8: return launch_cpl<T, 8, PACKED>(a, cpl, stream);
+        case 16: return launch_cpl<T, 16, PACKED>(a, cpl, stream);
+        default: return launch_cpl<T, 32, PACKED>(a, cpl, stream);
     }
 }
 
 template <bool PACKED>
 int32_t dispatch_dtype(int32_t dtype, const dcp::CombineArgs &a, cudaStream_t stream) {
-    constexpr int VW = PACKED ? 1 : 4;
     switch (dtype) {
-        case DCP_BF16: return dispatch_combine<dcp::Bf16, VW, PACKED>(a, stream);
-        case DCP_FP16: return dispatch_combine<dcp::Fp16, VW, PACKED>(a, stream);
-        default: return dispatch_combine<dcp::Fp32, VW, PACKED>(a, stream);
+        case DCP_BF16: return dispatch_combine<dcp::Bf16, PACKED>(a, stream);
+        case DCP_FP16: return dispatch_combine<dcp::Fp16, PACKED>(a, stream);
+        default: return dispatch_combine<dcp::Fp32, PACKED>(a, stream);
     }
 }
 
@@ -225,7 +297,8 @@ int32_t dcp_unpack_combine(const void *recv_buf, void *result, float *global_lse
     a.lse_stride_n = 0;
     a.data_w = (int32_t)(D * es / 4);
     a.row_pitch_w = a.data_w + 1;
-    a.chunks = a.data_w;
+    a.chunks = a.data_w / 4;
+    a.total_w = (int64_t)(N - 1) * a.shard_stride_w + a.units * a.row_pitch_w;
     a.N = N;
     a.base_e = is_lse_base_on_e ? 1 : 0;
     a.return_lse = return_lse ? 1 : 0;
@@ -267,18 +340,19 @@ int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_b
     a.src_stride_h_w = out_stride_h * es / 4;
     a.lse_stride_b = lse_stride_b;
     a.data_w = (int32_t)(D * es / 4);
-    a.chunks = a.data_w / 4;
-    a.chunks_magic = ((uint64_t(1) << 32) + (uint64_t)a.chunks - 1) / (uint64_t)a.chunks;
     a.row_pitch_w = a.data_w + 1;
-    // a tile of about 16 KiB of packed rows (at most one row per thread)
-    int tile_rows = 4096 / a.row_pitch_w;
-    if (tile_rows < 1) tile_rows = 1;
-    if (tile_rows > dcp::kPackThreads) tile_rows = dcp::kPackThreads;
-    a.tile_rows = tile_rows;
-    const size_t smem = (size_t)((3 + (int64_t)tile_rows * a.row_pitch_w + 3) / 4) * 16;
-
-    static const int per_sm = resident_ctas(dcp::pack_kernel, dcp::kPackThreads, 4 * 4096 + 64);
-    const int64_t tiles = (a.rows + tile_rows - 1) / tile_rows;
+    // a stage holds about 16 KiB of source rows (at least one) and their LSE
+    // words, plus 4 words of slack for the second aligned read of the last chunk
+    a.tile_rows = (dcp::kPackMinStageWords - 8) / a.row_pitch_w;
+    if (a.tile_rows < 1) a.tile_rows = 1;
+    a.stage_w = ((a.tile_rows * a.row_pitch_w + 3) & ~3) + 4;
+    a.pitch_magic = (uint32_t)(((uint64_t(1) << 32) + (uint64_t)a.row_pitch_w - 1) / (uint64_t)a.row_pitch_w);
+    const int chunks = a.data_w / 4;
+    a.lanes_per_row = chunks >= 32 ? 32 : chunks >= 16 ? 16 : chunks >= 8 ? 8 : 4;
+    const size_t smem = (size_t)dcp::kPackStages * a.stage_w * 4;
+    if (!pack_smem_reserved()) return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory for the pack kernel", fn);
+    const int per_sm = pack_resident_ctas(smem);
+    const int64_t tiles = (a.rows + a.tile_rows - 1) / a.tile_rows;
     const int64_t cap = (int64_t)sm_count() * per_sm;
     const int grid = (int)(tiles < cap ? tiles : cap);
     dcp::pack_kernel<<<grid, dcp::kPackThreads, smem, static_cast<cudaStream_t>(cuda_stream)>>>(a);

@@ -111,6 +111,25 @@ __device__ __forceinline__ uint32_t load_word(const uint32_t *p) {
     return r;
 }
 
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async_word(uint32_t *s, const uint32_t *g) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(s)), "l"(g) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_chunk(void *s, const uint32_t *g) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(s)), "l"(g) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int PENDING>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(PENDING) : "memory");
+}
+
 // An LSE that is NaN or +-inf becomes -inf; classified on the exponent bits so
 // the rule holds under any compiler math flags.
 __device__ __forceinline__ float sanitize_lse(uint32_t bits) {
@@ -142,31 +161,76 @@ struct CombineArgs {
     int64_t shard_stride_w;  // words between consecutive shards
     int64_t lse_stride_n;    // split layout: floats between consecutive shards
     int64_t row_pitch_w;     // words between consecutive rows of one shard
-    int32_t data_w;          // words of data per row (D * elemsize / 4)
-    int32_t chunks;          // data_w / VW
+    int64_t total_w;         // packed layout: words of the buffer that may be read
+    int32_t data_w;          // words of data per row (D * elemsize / 4), a multiple of 4
+    int32_t chunks;          // data_w / 4: 16-byte chunks per row
     int32_t slots;           // ceil(chunks / G): chunk slots per lane
     int32_t N;
     int32_t base_e;
     int32_t return_lse;
 };
 
-// One warp works on 32/G result rows at a time, G lanes per row.  Phase 1: the
-// G lanes of a row read the N LSEs (lane j takes shards j, j+G, ...), reduce
-// max and sum with shuffles, and leave the normalised weights in shared memory.
-// Phase 2: lane j accumulates chunks j, j+G, ... of the row over all N shards,
-// with NB shards' loads issued before their FMAs, and stores the rounded row.
-template <class T, int VW, int G, int CPL, int NB, bool PACKED>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineArgs a) {
+// The 4 words that start at word q (0..3) of the 8-word window (lo, hi).
+__device__ __forceinline__ Words<4> funnel_words(const Words<4> &lo, const Words<4> &hi, int q) {
+    uint32_t a0 = lo.w[0], a1 = lo.w[1], a2 = lo.w[2], a3 = lo.w[3], a4 = hi.w[0], a5 = hi.w[1], a6 = hi.w[2];
+    if (q & 2) {
+        a0 = a2; a1 = a3; a2 = a4; a3 = a5; a4 = a6;
+    }
+    if (q & 1) {
+        a0 = a1; a1 = a2; a2 = a3; a3 = a4;
+    }
+    Words<4> r;
+    r.w[0] = a0; r.w[1] = a1; r.w[2] = a2; r.w[3] = a3;
+    return r;
+}
+
+// The 16-byte chunk at word w of a 16-byte aligned buffer, reading no word at or
+// beyond `limit` (those come back as 0): the buffer's last row may end inside a chunk.
+__device__ __forceinline__ Words<4> load_chunk_bounded(const uint32_t *base, int64_t w, int64_t limit) {
+    if (w + 4 <= limit) return load_stream<4>(base + w);
+    Words<4> r;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) r.w[e] = (w + e < limit) ? load_word(base + w + e) : 0u;
+    return r;
+}
+
+// Shared memory of one combine CTA: per warp and per row in flight, the N
+// normalised weights, and (packed layout) the N tail chunks.
+__host__ __device__ constexpr size_t combine_smem_bytes(int units_per_warp, int N, bool packed) {
+    return (size_t)(kCombineThreads / 32) * units_per_warp * N * (sizeof(float) + (packed ? 16 : 0));
+}
+
+// One warp works on 32/G result rows at a time, G lanes per row; lane j of a row
+// owns its 16-byte chunks j, j+G, j+2G, ... (slots), CPL slots per pass.
+//   1. The loads of the first NB shards' chunks are issued.
+//   2. Phase 1 (weights): lane j takes shards j, j+G, ...; it reads each LSE
+//      (split: from the LSE array; packed: from the row's tail chunk, which it
+//      also keeps in shared memory), sanitises it by exponent bits, and the G
+//      lanes reduce max and sum with xor-shuffles.  The normalised weights go
+//      to shared memory; lane 0 writes the global LSE.
+//   3. Phase 2 (weighted sum): fp32 FMAs over all N shards, NB shards' loads
+//      in flight at a time, then one rounding and a 16-byte store per chunk.
+// Packed rows are 2D+4 bytes, so a row starts q = 0..3 words past a 16-byte
+// boundary.  Lanes load aligned chunks; output chunk c is the 4 words at offset
+// q of aligned chunks c and c+1, and aligned chunk c+1 comes from the next lane
+// by shuffle (lane G-1 takes lane 0's next slot), or from the tail chunk in
+// shared memory for the row's last chunk.
+template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS = 1>
+__global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(const CombineArgs a) {
     constexpr int kUnitsPerWarp = 32 / G;
     constexpr int kWarps = kCombineThreads / 32;
-    constexpr int kElems = VW * T::kPerWord;
-    __shared__ float s_w[kWarps][kUnitsPerWarp][kMaxShards];
+    constexpr int kElems = 4 * T::kPerWord;
+    extern __shared__ uint4 s_dyn[];
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int ul = lane / G;
     const int j = lane % G;
-    float *sw = s_w[warp][ul];
+    const int next_lane = (lane & ~(G - 1)) | ((j + 1) & (G - 1));
+    const int slot_base = warp * kUnitsPerWarp + ul;
+    uint4 *s_tail = s_dyn + (size_t)slot_base * a.N;  // packed only: [warps * units_per_warp][N]
+    float *sw = reinterpret_cast<float *>(s_dyn + (PACKED ? (size_t)kWarps * kUnitsPerWarp * a.N : 0)) +
+                (size_t)slot_base * a.N;
     const int64_t tasks = (a.units + kUnitsPerWarp - 1) / kUnitsPerWarp;
 
     for (int64_t task = (int64_t)blockIdx.x * kWarps + warp; task < tasks; task += (int64_t)gridDim.x * kWarps) {
@@ -174,14 +238,55 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
         const bool valid = u < a.units;
         const int64_t row = u * a.row_pitch_w;
 
+        int c[CPL];
+        bool act[CPL];
+        Words<4> x[NB][CPL];
+        int qv[NB];
+
+        auto set_pass = [&](int s0) {
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+                c[k] = j + G * (s0 + k);
+                act[k] = valid && c[k] < a.chunks;
+            }
+        };
+        auto issue = [&](int n0) {
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+                const int64_t w0 = (int64_t)(n0 + i) * a.shard_stride_w + row;
+                const int64_t wa = PACKED ? (w0 & ~int64_t(3)) : w0;
+                qv[i] = (int)(w0 & 3);
+#pragma unroll
+                for (int k = 0; k < CPL; ++k) {
+                    if (n0 + i < a.N && act[k]) {
+                        x[i][k] = load_stream<4>(a.src + wa + 4 * c[k]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) x[i][k].w[e] = 0u;
+                    }
+                }
+            }
+        };
+
+        set_pass(0);
+        issue(0);
+
         // ---- phase 1: weights of the N shards --------------------------------
         float lmax = -INFINITY;
         for (int n = j; n < a.N; n += G) {
             float l = -INFINITY;
             if (valid) {
-                const uint32_t bits =
-                    PACKED ? load_word(a.src + n * a.shard_stride_w + row + a.data_w)
-                           : load_word(reinterpret_cast<const uint32_t *>(a.lses) + n * a.lse_stride_n + u);
+                uint32_t bits;
+                if constexpr (PACKED) {
+                    const int64_t w0 = (int64_t)n * a.shard_stride_w + row;
+                    const int64_t wa = w0 & ~int64_t(3);
+                    const Words<4> t = load_chunk_bounded(a.src, wa + 4 * (int64_t)a.chunks, a.total_w);
+                    s_tail[n] = make_uint4(t.w[0], t.w[1], t.w[2], t.w[3]);
+                    const int q = (int)(w0 & 3);
+                    bits = q == 0 ? t.w[0] : q == 1 ? t.w[1] : q == 2 ? t.w[2] : t.w[3];
+                } else {
+                    bits = load_word(reinterpret_cast<const uint32_t *>(a.lses) + n * a.lse_stride_n + u);
+                }
                 l = sanitize_lse(bits);
             }
             sw[n] = l;
@@ -191,8 +296,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
         const float m = (lmax == -INFINITY) ? 0.0f : lmax;
         float wsum = 0.0f;
         for (int n = j; n < a.N; n += G) {
-            const float x = sw[n] - m;
-            float w = a.base_e ? expf(x) : exp2f(x);
+            const float x1 = sw[n] - m;
+            float w = a.base_e ? expf(x1) : exp2f(x1);
             if (w != w) w = 0.0f;
             sw[n] = w;
             wsum += w;
@@ -205,45 +310,49 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
 
         // ---- phase 2: weighted sum of the N rows -------------------------------
         for (int s0 = 0; s0 < a.slots; s0 += CPL) {
-            int c[CPL];
-            bool act[CPL];
+            if (s0 > 0) {
+                set_pass(s0);
+                issue(0);
+            }
             float acc[CPL][kElems];
 #pragma unroll
-            for (int k = 0; k < CPL; ++k) {
-                c[k] = j + G * (s0 + k);
-                act[k] = valid && c[k] < a.chunks;
+            for (int k = 0; k < CPL; ++k)
 #pragma unroll
                 for (int e = 0; e < kElems; ++e) acc[k][e] = 0.0f;
-            }
+            const bool more_passes = s0 + CPL < a.slots;
             for (int n0 = 0; n0 < a.N; n0 += NB) {
-                Words<VW> x[NB][CPL];
+                if (n0 > 0) issue(n0);
 #pragma unroll
                 for (int i = 0; i < NB; ++i) {
-                    const int64_t base = (int64_t)(n0 + i) * a.shard_stride_w + row;
+                    if (n0 + i >= a.N) break;  // uniform across the warp
+                    const int n = n0 + i;
+                    const float w = sw[n];
 #pragma unroll
                     for (int k = 0; k < CPL; ++k) {
-                        if (n0 + i < a.N && act[k]) {
-                            x[i][k] = load_stream<VW>(a.src + base + (int64_t)c[k] * VW);
-                        } else {
+                        Words<4> v = x[i][k];
+                        if constexpr (PACKED) {
+                            // aligned chunk c+1: lane j+1's slot k, or lane 0's slot k+1 for lane G-1
+                            Words<4> send = x[i][k];
+                            if (k + 1 < CPL && j == 0) send = x[i][k + 1];
+                            Words<4> nx;
 #pragma unroll
-                            for (int v = 0; v < VW; ++v) x[i][k].w[v] = 0u;
-                        }
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < NB; ++i) {
-                    if (n0 + i < a.N) {
-                        const float w = sw[n0 + i];
-#pragma unroll
-                        for (int k = 0; k < CPL; ++k) {
-#pragma unroll
-                            for (int v = 0; v < VW; ++v) {
-                                float f[T::kPerWord];
-                                T::decode(x[i][k].w[v], f);
-#pragma unroll
-                                for (int e = 0; e < T::kPerWord; ++e)
-                                    acc[k][v * T::kPerWord + e] = fmaf(w, f[e], acc[k][v * T::kPerWord + e]);
+                            for (int e = 0; e < 4; ++e) nx.w[e] = __shfl_sync(0xffffffffu, send.w[e], next_lane);
+                            if (act[k] && c[k] == a.chunks - 1) {
+                                const uint4 t = s_tail[n];
+                                nx.w[0] = t.x; nx.w[1] = t.y; nx.w[2] = t.z; nx.w[3] = t.w;
+                            } else if (act[k] && k == CPL - 1 && j == G - 1 && more_passes) {
+                                const int64_t wa = ((int64_t)n * a.shard_stride_w + row) & ~int64_t(3);
+                                nx = load_stream<4>(a.src + wa + 4 * (c[k] + 1));
                             }
+                            v = funnel_words(v, nx, qv[i]);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float f[T::kPerWord];
+                            T::decode(v.w[e], f);
+#pragma unroll
+                            for (int h = 0; h < T::kPerWord; ++h)
+                                acc[k][e * T::kPerWord + h] = fmaf(w, f[h], acc[k][e * T::kPerWord + h]);
                         }
                     }
                 }
@@ -251,10 +360,10 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
 #pragma unroll
             for (int k = 0; k < CPL; ++k) {
                 if (act[k]) {
-                    Words<VW> o;
+                    Words<4> o;
 #pragma unroll
-                    for (int v = 0; v < VW; ++v) o.w[v] = T::encode(&acc[k][v * T::kPerWord]);
-                    store_words<VW>(a.result + u * a.data_w + (int64_t)c[k] * VW, o);
+                    for (int e = 0; e < 4; ++e) o.w[e] = T::encode(&acc[k][e * T::kPerWord]);
+                    store_words<4>(a.result + u * a.data_w + 4 * (int64_t)c[k], o);
                 }
             }
         }
@@ -264,107 +373,180 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineA
 
 // ---------------------------------------------------------------------------
 // pack
+constexpr int kPackStages = 4;            // shared-memory tiles in flight per CTA
+constexpr int kPackMinStageWords = 4096;  // 16 KiB per tile (more when one row needs it)
+
 struct PackArgs {
     const uint32_t *src;      // cp_attn_out as words
     const uint32_t *lse;      // cp_attn_lse as raw 32-bit words
-    uint32_t *dst;            // send buffer as words
+    uint32_t *dst;            // send buffer as words (16-byte aligned)
     int64_t rows;             // N * B * Hr packed rows
     int64_t B;
     int64_t Hr;
     int64_t src_stride_b_w;   // words between tokens of cp_attn_out
     int64_t src_stride_h_w;   // words between heads of cp_attn_out
     int64_t lse_stride_b;     // words between tokens of cp_attn_lse
-    int32_t data_w;           // words of data per row
-    int32_t chunks;           // data_w / 4 (16-byte chunks per source row)
-    uint64_t chunks_magic;    // ceil(2^32 / chunks): n / chunks == (n * magic) >> 32 whenever n * chunks < 2^32
-    int32_t row_pitch_w;      // data_w + 1
+    uint32_t pitch_magic;     // ceil(2^32 / row_pitch_w): t / row_pitch_w == umulhi(t, magic) when t * row_pitch_w < 2^32
+    int32_t data_w;           // words of data per row (a multiple of 4)
+    int32_t row_pitch_w;      // data_w + 1: words per packed row
     int32_t tile_rows;        // packed rows per tile
+    int32_t stage_w;          // words per shared-memory stage (a multiple of 4)
+    int32_t lanes_per_row;    // 4, 8, 16 or 32 lanes copy one source row
 };
 
-// A CTA packs tiles of `tile_rows` consecutive packed rows, i.e. one contiguous
-// word range of the send buffer.  It gathers the source rows (16-byte loads)
-// and their LSE words into shared memory laid out exactly as that range, with
-// the same alignment modulo 16 bytes, then writes the range back with 16-byte
-// stores (4-byte stores only for the partial chunks at its two ends).  Every
-// word of the send buffer is written once, by one CTA.
+// (rank, token, head) of packed row i: rows are ordered [rank][token][head].
+__device__ __forceinline__ void pack_row_coords(int64_t i, int64_t B, int64_t Hr, int64_t &rank, int64_t &b,
+                                                int64_t &h) {
+    const int64_t per_rank = B * Hr;
+    if (i < (int64_t(1) << 32) && per_rank < (int64_t(1) << 32)) {
+        const uint32_t i32 = (uint32_t)i, pr = (uint32_t)per_rank, hr = (uint32_t)Hr;
+        const uint32_t r = i32 / pr, rem = i32 - r * pr, bb = rem / hr;
+        rank = r;
+        b = bb;
+        h = rem - bb * hr;
+    } else {
+        rank = i / per_rank;
+        const int64_t rem = i - rank * per_rank;
+        b = rem / Hr;
+        h = rem - b * Hr;
+    }
+}
+
+// A CTA packs tiles of `tile_rows` consecutive packed rows (one contiguous word
+// range of the send buffer), kPackStages tiles in flight.
+//   Loads: the tile's source rows (16-byte aligned, whole 16-byte chunks) are
+//   copied with 16-byte cp.async into a stage, row after row, and each row's
+//   LSE word into a small array behind them.
+//   Stores, once a tile has landed: packed word t of the tile is row
+//   r = t / (D'+1), word k = t mod (D'+1) (D' = data words per row), i.e. stage
+//   word t - r when k < D', else LSE r.  Pass 1 writes every whole 16-byte
+//   chunk that lies inside one row's data: two aligned 16-byte shared loads and
+//   a word funnel.  Pass 2 writes, one thread per row, the chunk that holds the
+//   row's LSE word (rows are >= 5 words, so a chunk holds at most one LSE).
+//   The partial chunks at the two ends of the range use 4-byte stores.
+// Every word of the send buffer is written once, by one CTA.
 __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a) {
-    extern __shared__ uint4 s_tile_v4[];
-    uint32_t *s_tile = reinterpret_cast<uint32_t *>(s_tile_v4);
-    __shared__ int64_t s_src_row[kPackThreads];
-
+    extern __shared__ uint4 s_stage_v4[];
+    uint32_t *s_stage = reinterpret_cast<uint32_t *>(s_stage_v4);
+    constexpr int kWarps = kPackThreads / 32;
     const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
     const int64_t tiles = (a.rows + a.tile_rows - 1) / a.tile_rows;
-    const int64_t per_rank = a.B * a.Hr;
+    const int64_t my_tiles = tiles > blockIdx.x ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int lse_base = a.tile_rows * a.data_w;  // LSE words follow the rows in a stage
+    const int chunks = a.data_w >> 2;
 
-    for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    // copies of this CTA's k-th tile into stage k % kPackStages
+    auto issue = [&](int64_t k) {
+        const int64_t tile = blockIdx.x + k * gridDim.x;
         const int64_t i0 = tile * a.tile_rows;
         const int nrows = (int)min((int64_t)a.tile_rows, a.rows - i0);
-        const int64_t dst_w0 = i0 * a.row_pitch_w;
-        const int q = (int)(dst_w0 & 3);  // alignment of the range start, in words
-
-        // source row offsets and LSE words, one thread per packed row
-        for (int r = tid; r < nrows; r += kPackThreads) {
-            const int64_t i = i0 + r;
-            const int64_t rank = i / per_rank;
-            const int64_t rem = i - rank * per_rank;
-            const int64_t b = rem / a.Hr;
-            const int64_t head = rank * a.Hr + (rem - b * a.Hr);
-            s_src_row[r] = b * a.src_stride_b_w + head * a.src_stride_h_w;
-            s_tile[q + r * a.row_pitch_w + a.data_w] = load_word(a.lse + b * a.lse_stride_b + head);
+        uint32_t *stage = s_stage + (int)(k % kPackStages) * a.stage_w;
+        // warp w copies rows [r0, r1) of the tile, 32 / lpr rows at a time
+        const int r0 = (nrows * warp) / kWarps;
+        const int r1 = (nrows * (warp + 1)) / kWarps;
+        const int lpr = a.lanes_per_row;
+        const int rpi = 32 / lpr;
+        const int sub = lane % lpr;
+        int r = r0 + lane / lpr;
+        if (r >= r1) return;
+        int64_t rank, b, h;
+        pack_row_coords(i0 + r, a.B, a.Hr, rank, b, h);
+        for (;;) {
+            const int64_t head = rank * a.Hr + h;
+            const uint32_t *src = a.src + b * a.src_stride_b_w + head * a.src_stride_h_w;
+            uint32_t *srow = stage + r * a.data_w;
+            for (int c = sub; c < chunks; c += lpr) cp_async_chunk(srow + 4 * c, src + 4 * c);
+            if (sub == 0) cp_async_word(stage + lse_base + r, a.lse + b * a.lse_stride_b + head);
+            r += rpi;
+            if (r >= r1) break;
+            h += rpi;
+            while (h >= a.Hr) {
+                h -= a.Hr;
+                if (++b == a.B) {
+                    b = 0;
+                    ++rank;
+                }
+            }
         }
-        __syncthreads();
+    };
 
-        // gather: 16-byte loads from the source rows, 4-byte shared stores; the
-        // store order is rotated by lane/8 so the 32 lanes hit 32 distinct banks
-        const int total_chunks = nrows * a.chunks;
-        const int rot = (tid >> 3) & 3;
-        for (int idx = tid; idx < total_chunks; idx += kPackThreads) {
-            const int r = (int)(((uint64_t)idx * a.chunks_magic) >> 32);
-            const int c = idx - r * a.chunks;
-            const Words<4> v = load_stream<4>(a.src + s_src_row[r] + 4 * c);
-            uint32_t *s = s_tile + q + r * a.row_pitch_w + 4 * c;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int e = (k + rot) & 3;
-                const uint32_t val = e == 0 ? v.w[0] : e == 1 ? v.w[1] : e == 2 ? v.w[2] : v.w[3];
-                s[e] = val;
-            }
-        }
-        __syncthreads();
-
-        // scatter: shared word s <-> send-buffer word dst_w0 - q + s
-        const int end = q + nrows * a.row_pitch_w;  // one past the last shared word in use
-        uint32_t *dst = a.dst + (dst_w0 - q);
-        const int first_full = q ? 1 : 0;           // first 16-byte chunk fully inside the range
-        const int full_end = end >> 2;              // one past the last full chunk
-        for (int t = first_full + tid; t < full_end; t += kPackThreads) {
-            const uint4 v = s_tile_v4[t];
-            Words<4> o;
-            o.w[0] = v.x;
-            o.w[1] = v.y;
-            o.w[2] = v.z;
-            o.w[3] = v.w;
-            store_words<4>(dst + 4 * t, o);
-        }
-        // A range holds at least one packed row of >= 5 words, so end >= 5: the
-        // head words [q, 4) and the tail words [4 * full_end, end) never overlap.
-        if (tid < 4) {  // the partial chunk at the head of the range
-            const int s = tid;
-            if (s >= q && q > 0) {
-                Words<1> o;
-                o.w[0] = s_tile[s];
-                store_words<1>(dst + s, o);
-            }
-        } else if (tid < 8) {  // the partial chunk at the tail
-            const int s = 4 * full_end + (tid - 4);
-            if (s < end) {
-                Words<1> o;
-                o.w[0] = s_tile[s];
-                store_words<1>(dst + s, o);
-            }
-        }
-        __syncthreads();
+    for (int k = 0; k < kPackStages - 1; ++k) {
+        if (k < my_tiles) issue(k);
+        cp_async_commit();
     }
+    for (int64_t k = 0; k < my_tiles; ++k) {
+        if (k + kPackStages - 1 < my_tiles) issue(k + kPackStages - 1);
+        cp_async_commit();
+        cp_async_wait<kPackStages - 1>();  // this thread's copies of tile k have landed
+        __syncthreads();                   // ... and everyone else's
+
+        const int64_t tile = blockIdx.x + k * gridDim.x;
+        const int64_t i0 = tile * a.tile_rows;
+        const int nrows = (int)min((int64_t)a.tile_rows, a.rows - i0);
+        const int64_t d0 = i0 * a.row_pitch_w;  // first send word of the tile
+        const int len = nrows * a.row_pitch_w;
+        const uint32_t *stage = s_stage + (int)(k % kPackStages) * a.stage_w;
+        const uint4 *stage_v4 = reinterpret_cast<const uint4 *>(stage);
+        auto word_of = [&](int r, int kk) -> uint32_t {  // word kk of packed row r of the tile
+            return kk < a.data_w ? stage[r * a.data_w + kk] : stage[lse_base + r];
+        };
+        const int lead = (int)((4 - (d0 & 3)) & 3);  // words before the first 16-byte boundary
+        const int full = (len - lead) >> 2;           // whole 16-byte chunks of the range
+        uint32_t *dst_full = a.dst + d0 + lead;       // 16-byte aligned; chunk g = words lead+4g .. +3
+
+        // pass 1: chunks inside one row's data
+        for (int g = tid; g < full; g += kPackThreads) {
+            const int t0 = lead + 4 * g;
+            const int r = (int)__umulhi((uint32_t)t0, a.pitch_magic);
+            const int kk = t0 - r * a.row_pitch_w;
+            if (kk + 3 < a.data_w) {
+                const int base = t0 - r;  // stage word of packed word t0
+                const uint4 lo4 = stage_v4[base >> 2];
+                const uint4 hi4 = stage_v4[(base >> 2) + 1];
+                Words<4> lo, hi;
+                lo.w[0] = lo4.x; lo.w[1] = lo4.y; lo.w[2] = lo4.z; lo.w[3] = lo4.w;
+                hi.w[0] = hi4.x; hi.w[1] = hi4.y; hi.w[2] = hi4.z; hi.w[3] = hi4.w;
+                store_words<4>(dst_full + 4 * g, funnel_words(lo, hi, base & 3));
+            }
+        }
+        // pass 2: the chunk holding each row's LSE word
+        for (int r = tid; r < nrows; r += kPackThreads) {
+            const int t_row = r * a.row_pitch_w;
+            const int t_lse = t_row + a.data_w;
+            const int g = (t_lse - lead) >> 2;
+            if (t_lse >= lead && g < full) {
+                Words<4> o;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int kk = lead + 4 * g + e - t_row;
+                    o.w[e] = kk < a.row_pitch_w ? word_of(r, kk) : word_of(r + 1, kk - a.row_pitch_w);
+                }
+                store_words<4>(dst_full + 4 * g, o);
+            }
+        }
+        // the partial chunks at the two ends of the range (a range has >= 5 words)
+        auto word_at = [&](int t) -> uint32_t {
+            const int r = (int)__umulhi((uint32_t)t, a.pitch_magic);
+            return word_of(r, t - r * a.row_pitch_w);
+        };
+        if (tid < lead) {
+            Words<1> o;
+            o.w[0] = word_at(tid);
+            store_words<1>(a.dst + d0 + tid, o);
+        } else if (tid >= 4 && tid < 8) {
+            const int t = lead + 4 * full + (tid - 4);
+            if (t < len) {
+                Words<1> o;
+                o.w[0] = word_at(t);
+                store_words<1>(a.dst + d0 + t, o);
+            }
+        }
+        __syncthreads();  // stage k % kPackStages is free for tile k + kPackStages
+    }
+    cp_async_wait<0>();
 }
 
 }  // namespace dcp

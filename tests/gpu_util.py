@@ -23,6 +23,13 @@ def raw(t: torch.Tensor) -> np.ndarray:
     return t.numpy()
 
 
+def bits(a) -> np.ndarray:
+    """Integer view of a tensor's or array's elements (uint16 / uint32), for bit-exact comparison."""
+    if isinstance(a, torch.Tensor):
+        a = raw(a)
+    return a.view(np.uint32) if a.dtype.itemsize == 4 else a.view(np.uint16)
+
+
 def as_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().to(torch.float64).numpy()
 
