@@ -131,10 +131,10 @@ int cached_resident_ctas(K kernel, InstanceCache &ic, int threads, size_t smem) 
     return n;
 }
 
-template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS>
+template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS, bool UNIFORM>
 int32_t launch_combine(const dcp::CombineArgs &a, cudaStream_t stream) {
     const char *fn = PACKED ? "dcp_unpack_combine" : "dcp_lse_combine";
-    auto kernel = dcp::combine_kernel<T, G, CPL, NB, PACKED, MIN_CTAS>;
+    auto kernel = dcp::combine_kernel<T, G, CPL, NB, PACKED, MIN_CTAS, UNIFORM>;
     static InstanceCache ic;
     constexpr int kUnitsPerWarp = 32 / G;
     constexpr int kWarps = dcp::kCombineThreads / 32;
@@ -154,35 +154,49 @@ int32_t launch_combine(const dcp::CombineArgs &a, cudaStream_t stream) {
 // bytes in flight per SM are set by how many warps fit.  Capping registers so
 // that 3 CTAs fit (2 for the four-slot shapes, which spill otherwise) measured
 // best on B200 for every shape.
-template <class T, int G, bool PACKED>
+template <class T, int G, bool PACKED, bool UNIFORM>
 int32_t launch_cpl(dcp::CombineArgs a, int cpl, cudaStream_t stream) {
     switch (cpl) {
-        case 1: return launch_combine<T, G, 1, 8, PACKED, 3>(a, stream);
-        case 2: return launch_combine<T, G, 2, 4, PACKED, 3>(a, stream);
-        default: return launch_combine<T, G, 4, 2, PACKED, 2>(a, stream);
+        case 1: return launch_combine<T, G, 1, 8, PACKED, 3, UNIFORM>(a, stream);
+        case 2: return launch_combine<T, G, 2, 4, PACKED, 3, UNIFORM>(a, stream);
+        default: return launch_combine<T, G, 4, 2, PACKED, 2, UNIFORM>(a, stream);
+    }
+}
+
+template <class T, bool PACKED, bool UNIFORM>
+int32_t launch_g(dcp::CombineArgs a, int G, int cpl, cudaStream_t stream) {
+    switch (G) {
+        case 4: return launch_cpl<T, 4, PACKED, UNIFORM>(a, cpl, stream);
+        case 8: return launch_cpl<T, 8, PACKED, UNIFORM>(a, cpl, stream);
+        case 16: return launch_cpl<T, 16, PACKED, UNIFORM>(a, cpl, stream);
+        default: return launch_cpl<T, 32, PACKED, UNIFORM>(a, cpl, stream);
     }
 }
 
 // Shape of the work per lane.  Each lane should keep about eight 16-byte loads
 // in flight: chunk slots per lane (CPL) times shards per batch (NB = 8 / CPL),
 // so fewer shards ask for more chunks per lane, i.e. fewer lanes per row (G).
-// The packed layout never goes below two slots per lane: its per-shard
-// realignment favours fewer, longer lane groups.
+// When all shards of the packed buffer put a row at the same offset from a
+// 16-byte boundary (the shard stride is a multiple of 16 bytes) and one pass
+// covers a row, the sums are realigned once per output chunk ("uniform");
+// otherwise every shard's chunk is realigned, and that path keeps at least two
+// slots per lane.
 template <class T, bool PACKED>
 int32_t dispatch_combine(dcp::CombineArgs a, cudaStream_t stream) {
     const int chunks = a.chunks;
+    const bool uniform = PACKED && (a.N == 1 || a.shard_stride_w % 4 == 0) && chunks <= 4 * 32;
     int cpl_target = a.N >= 8 ? 1 : a.N >= 4 ? 2 : 4;
-    if (PACKED && cpl_target < 2) cpl_target = 2;
+    if (PACKED && !uniform && cpl_target < 2) cpl_target = 2;
     const int per_lane = (chunks + cpl_target - 1) / cpl_target;
     int G = 4;
     while (G < per_lane && G < 32) G *= 2;
     a.slots = (chunks + G - 1) / G;
-    const int cpl = a.slots >= 3 ? 4 : a.slots;
-    switch (G) {
-        case 4: return launch_cpl<T, 4, PACKED>(a, cpl, stream);
-        case 8: return launch_cpl<T, 8, PACKED>(a, cpl, stream);
-        case 16: return launch_cpl<T, 16, PACKED>(a, cpl, stream);
-        default: return launch_cpl<T, 32, PACKED>(a, cpl, stream);
+    const int cpl = a.slots >= 3 ? 4 : a.slots;  // one pass whenever slots <= 4
+    if constexpr (PACKED) {
+        if (uniform) return launch_g<T, true, true>(a, G, cpl, stream);
+        return launch_g<T, true, false>(a, G, cpl, stream);
+    } else {
+        return launch_g<T, false, false>(a, G, cpl, stream);
     }
 }
 

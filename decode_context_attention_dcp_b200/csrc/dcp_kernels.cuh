@@ -215,7 +215,13 @@ __host__ __device__ constexpr size_t combine_smem_bytes(int units_per_warp, int 
 // q of aligned chunks c and c+1, and aligned chunk c+1 comes from the next lane
 // by shuffle (lane G-1 takes lane 0's next slot), or from the tail chunk in
 // shared memory for the row's last chunk.
-template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS = 1>
+// UNIFORM (packed, every shard's rows at the same offset q -- shard strides a
+// multiple of 16 bytes -- and one pass): the lanes accumulate the aligned chunks
+// as they are, and only the fp32 sums are realigned, once per output chunk:
+// output chunk c is elements 2q/e.. of sum c and the first ones of sum c+1 (from
+// the next lane, or, for the last chunk, the weighted sum of the tail chunks,
+// formed in phase 1 and reduced over the lane group).
+template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS = 1, bool UNIFORM = false>
 __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(const CombineArgs a) {
     constexpr int kUnitsPerWarp = 32 / G;
     constexpr int kWarps = kCombineThreads / 32;
@@ -306,6 +312,29 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
         const float denom = fmaxf(wsum, 1e-10f);
         for (int n = j; n < a.N; n += G) sw[n] = sw[n] / denom;
         if (a.return_lse && valid && j == 0) a.glse[u] = (a.base_e ? logf(wsum) : log2f(wsum)) + m;
+
+        // UNIFORM: weighted sum of the shards' tail chunks, reduced over the lane group
+        float tacc[kElems];
+        if constexpr (PACKED && UNIFORM) {
+#pragma unroll
+            for (int e = 0; e < kElems; ++e) tacc[e] = 0.0f;
+            for (int n = j; n < a.N; n += G) {
+                const uint4 t = s_tail[n];
+                const float w = sw[n];
+                const uint32_t tw[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float f[T::kPerWord];
+                    T::decode(tw[e], f);
+#pragma unroll
+                    for (int h = 0; h < T::kPerWord; ++h)
+                        tacc[e * T::kPerWord + h] = fmaf(w, f[h], tacc[e * T::kPerWord + h]);
+                }
+            }
+            // only the first 3 words (the most a row can leave in its tail chunk) matter
+#pragma unroll
+            for (int e = 0; e < 3 * T::kPerWord; ++e) tacc[e] = group_sum<G>(tacc[e]);
+        }
         __syncwarp();
 
         // ---- phase 2: weighted sum of the N rows -------------------------------
@@ -330,7 +359,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
 #pragma unroll
                     for (int k = 0; k < CPL; ++k) {
                         Words<4> v = x[i][k];
-                        if constexpr (PACKED) {
+                        if constexpr (PACKED && !UNIFORM) {
                             // aligned chunk c+1: lane j+1's slot k, or lane 0's slot k+1 for lane G-1
                             Words<4> send = x[i][k];
                             if (k + 1 < CPL && j == 0) send = x[i][k + 1];
@@ -357,13 +386,52 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
                     }
                 }
             }
+            if constexpr (PACKED && UNIFORM) {
+                // sum c+1 for output chunk c: the next lane's slot k, lane 0's slot k+1 for
+                // lane G-1, the tail sum for the row's last chunk
+                const int q = qv[0];  // the same for every shard
 #pragma unroll
-            for (int k = 0; k < CPL; ++k) {
-                if (act[k]) {
-                    Words<4> o;
+                for (int k = 0; k < CPL; ++k) {
+                    float nx[kElems];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) o.w[e] = T::encode(&acc[k][e * T::kPerWord]);
-                    store_words<4>(a.result + u * a.data_w + 4 * (int64_t)c[k], o);
+                    for (int e = 0; e < 3 * T::kPerWord; ++e) {
+                        const float send = (k + 1 < CPL && j == 0) ? acc[k + 1 < CPL ? k + 1 : k][e] : acc[k][e];
+                        nx[e] = __shfl_sync(0xffffffffu, send, next_lane);
+                    }
+                    if (act[k] && c[k] == a.chunks - 1) {
+#pragma unroll
+                        for (int e = 0; e < 3 * T::kPerWord; ++e) nx[e] = tacc[e];
+                    }
+                    if (act[k]) {
+                        // elements from word q of sum c, then the first words of sum c+1
+                        float outv[kElems];
+#pragma unroll
+                        for (int e = 0; e < kElems; ++e) {
+                            float v = 0.0f;
+#pragma unroll
+                            for (int qq = 0; qq < 4; ++qq) {
+                                const int s2 = e + qq * T::kPerWord;
+                                const float cand = s2 < kElems ? acc[k][s2 < kElems ? s2 : 0]
+                                                               : nx[s2 - kElems < 3 * T::kPerWord ? s2 - kElems : 0];
+                                if (qq == q) v = cand;
+                            }
+                            outv[e] = v;
+                        }
+                        Words<4> o;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o.w[e] = T::encode(&outv[e * T::kPerWord]);
+                        store_words<4>(a.result + u * a.data_w + 4 * (int64_t)c[k], o);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < CPL; ++k) {
+                    if (act[k]) {
+                        Words<4> o;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o.w[e] = T::encode(&acc[k][e * T::kPerWord]);
+                        store_words<4>(a.result + u * a.data_w + 4 * (int64_t)c[k], o);
+                    }
                 }
             }
         }

@@ -211,8 +211,10 @@ def _case(N, B, Hr, D, dtype, seed, p_neginf=0.1, p_nan=0.05, base_e=True):
 EDGE = [(N, B, Hr, D, dt)
         for (N, B, Hr, D) in [(1, 3, 2, 128), (2, 1, 1, 8), (3, 37, 3, 64), (5, 7, 5, 96), (16, 9, 2, 512),
                               (64, 3, 2, 128), (7, 2, 3, 576), (4, 5, 1, 1024), (2, 129, 4, 16), (33, 4, 3, 256),
-                              # rows too wide for shared-memory staging: the register-streaming kernel
-                              (64, 2, 2, 1024), (33, 3, 2, 1024), (40, 2, 1, 2048), (9, 300, 1, 8192)]
+                              # wide rows: several chunk slots per lane, several passes
+                              (64, 2, 2, 1024), (33, 3, 2, 1024), (40, 2, 1, 2048), (9, 300, 1, 8192),
+                              # packed rows at every offset from a 16-byte boundary in one shard stride
+                              (3, 8, 4, 576), (5, 4, 4, 96), (12, 16, 2, 64)]
         for dt in ("bf16", "fp16", "fp32")]
 
 
