@@ -69,6 +69,13 @@ int resident_ctas(K kernel, int threads, size_t smem) {
     return n;
 }
 
+// ceil(2^64 / d) for d >= 2; 0 stands for d == 1 (n / 1 == n).
+uint64_t magic64(uint64_t d) {
+    if (d <= 1) return 0;
+    const unsigned __int128 one = 1;
+    return (uint64_t)(((one << 64) + d - 1) / d);
+}
+
 // The pack kernel's dynamic shared memory can exceed the default 48 KiB: opt in
 // once per device, for the largest stage any accepted row width needs.
 bool pack_smem_reserved() {
@@ -359,9 +366,14 @@ int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_b
     // words, plus 4 words of slack for the second aligned read of the last chunk
     a.tile_rows = (dcp::kPackMinStageWords - 8) / a.row_pitch_w;
     if (a.tile_rows < 1) a.tile_rows = 1;
+    if (a.tile_rows > dcp::kPackMaxTileRows) a.tile_rows = dcp::kPackMaxTileRows;
     a.stage_w = ((a.tile_rows * a.row_pitch_w + 3) & ~3) + 4;
+    if (a.rows >= (int64_t(1) << 32))
+        return fail(DCP_ERR_INVALID_ARG, "%s: more than 2^32 packed rows", fn);
+    a.per_rank_magic = magic64((uint64_t)(B * a.Hr));
+    a.hr_magic = magic64((uint64_t)a.Hr);
     a.pitch_magic = (uint32_t)(((uint64_t(1) << 32) + (uint64_t)a.row_pitch_w - 1) / (uint64_t)a.row_pitch_w);
-    const int chunks = a.data_w / 4;
+    const uint64_t chunks = (uint64_t)a.data_w / 4;
     a.lanes_per_row = chunks >= 32 ? 32 : chunks >= 16 ? 16 : chunks >= 8 ? 8 : 4;
     const size_t smem = (size_t)dcp::kPackStages * a.stage_w * 4;
     if (!pack_smem_reserved()) return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory for the pack kernel", fn);

@@ -93,16 +93,18 @@ __device__ __forceinline__ Words<1> load_stream<1>(const uint32_t *p) {
 template <int VW>
 __device__ __forceinline__ void store_words(uint32_t *p, const Words<VW> &v);
 
+// Stores carry no "memory" clobber: nothing in these kernels reads what they
+// write, and a clobber would make the compiler reload every kernel argument
+// after each store.
 template <>
 __device__ __forceinline__ void store_words<4>(uint32_t *p, const Words<4> &v) {
     asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]),
-                 "r"(v.w[3])
-                 : "memory");
+                 "r"(v.w[3]));
 }
 
 template <>
 __device__ __forceinline__ void store_words<1>(uint32_t *p, const Words<1> &v) {
-    asm volatile("st.global.u32 [%0], %1;" ::"l"(p), "r"(v.w[0]) : "memory");
+    asm volatile("st.global.u32 [%0], %1;" ::"l"(p), "r"(v.w[0]));
 }
 
 __device__ __forceinline__ uint32_t load_word(const uint32_t *p) {
@@ -115,12 +117,15 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Asynchronous copies into shared memory.  They need no "memory" clobber: reads
+// of the copied words are ordered by cp.async.wait_group (which has one) and the
+// barrier after it.
 __device__ __forceinline__ void cp_async_word(uint32_t *s, const uint32_t *g) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(s)), "l"(g) : "memory");
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(s)), "l"(g));
 }
 
 __device__ __forceinline__ void cp_async_chunk(void *s, const uint32_t *g) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(s)), "l"(g) : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(s)), "l"(g));
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -443,6 +448,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
 // pack
 constexpr int kPackStages = 4;            // shared-memory tiles in flight per CTA
 constexpr int kPackMinStageWords = 4096;  // 16 KiB per tile (more when one row needs it)
+constexpr int kPackMaxTileRows = 64;      // rows per tile (row tables in shared memory)
 
 struct PackArgs {
     const uint32_t *src;      // cp_attn_out as words
@@ -454,112 +460,118 @@ struct PackArgs {
     int64_t src_stride_b_w;   // words between tokens of cp_attn_out
     int64_t src_stride_h_w;   // words between heads of cp_attn_out
     int64_t lse_stride_b;     // words between tokens of cp_attn_lse
+    uint64_t per_rank_magic;  // ceil(2^64 / (B * Hr)), 0 when B * Hr == 1
+    uint64_t hr_magic;        // ceil(2^64 / Hr), 0 when Hr == 1
     uint32_t pitch_magic;     // ceil(2^32 / row_pitch_w): t / row_pitch_w == umulhi(t, magic) when t * row_pitch_w < 2^32
+    int32_t lanes_per_row;    // lanes that copy one source row: 4, 8, 16 or 32
     int32_t data_w;           // words of data per row (a multiple of 4)
     int32_t row_pitch_w;      // data_w + 1: words per packed row
     int32_t tile_rows;        // packed rows per tile
     int32_t stage_w;          // words per shared-memory stage (a multiple of 4)
-    int32_t lanes_per_row;    // 4, 8, 16 or 32 lanes copy one source row
 };
 
-// (rank, token, head) of packed row i: rows are ordered [rank][token][head].
-__device__ __forceinline__ void pack_row_coords(int64_t i, int64_t B, int64_t Hr, int64_t &rank, int64_t &b,
-                                                int64_t &h) {
-    const int64_t per_rank = B * Hr;
-    if (i < (int64_t(1) << 32) && per_rank < (int64_t(1) << 32)) {
-        const uint32_t i32 = (uint32_t)i, pr = (uint32_t)per_rank, hr = (uint32_t)Hr;
-        const uint32_t r = i32 / pr, rem = i32 - r * pr, bb = rem / hr;
-        rank = r;
-        b = bb;
-        h = rem - bb * hr;
-    } else {
-        rank = i / per_rank;
-        const int64_t rem = i - rank * per_rank;
-        b = rem / Hr;
-        h = rem - b * Hr;
-    }
+// n / d for n < 2^32 and d <= 2^32, with magic = ceil(2^64 / d) (0 meaning d == 1).
+__device__ __forceinline__ uint64_t div_magic(uint64_t n, uint64_t magic) {
+    return magic ? __umul64hi(n, magic) : n;
 }
 
 // A CTA packs tiles of `tile_rows` consecutive packed rows (one contiguous word
 // range of the send buffer), kPackStages tiles in flight.
+//   Row table: for each tile, one thread per row computes the row's source
+//   offset and LSE index (one tile ahead of its copies).
 //   Loads: the tile's source rows (16-byte aligned, whole 16-byte chunks) are
-//   copied with 16-byte cp.async into a stage, row after row, and each row's
-//   LSE word into a small array behind them.
+//   copied with 16-byte cp.async into a stage, row after row, a group of lanes
+//   per row; each row's LSE word goes behind the rows.
 //   Stores, once a tile has landed: packed word t of the tile is row
 //   r = t / (D'+1), word k = t mod (D'+1) (D' = data words per row), i.e. stage
 //   word t - r when k < D', else LSE r.  Pass 1 writes every whole 16-byte
-//   chunk that lies inside one row's data: two aligned 16-byte shared loads and
-//   a word funnel.  Pass 2 writes, one thread per row, the chunk that holds the
-//   row's LSE word (rows are >= 5 words, so a chunk holds at most one LSE).
+//   chunk that lies inside one row's data as two aligned 16-byte shared loads
+//   and a word funnel.  Pass 2 writes, one thread per row, the chunk that holds
+//   the row's LSE word (rows are >= 5 words, so a chunk holds at most one LSE).
 //   The partial chunks at the two ends of the range use 4-byte stores.
 // Every word of the send buffer is written once, by one CTA.
 __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a) {
     extern __shared__ uint4 s_stage_v4[];
     uint32_t *s_stage = reinterpret_cast<uint32_t *>(s_stage_v4);
-    constexpr int kWarps = kPackThreads / 32;
+    __shared__ int64_t s_row_src[kPackStages][kPackMaxTileRows];  // word offset of each source row
+    __shared__ int64_t s_row_lse[kPackStages][kPackMaxTileRows];  // index of each row's LSE
     const int tid = threadIdx.x;
-    const int lane = tid & 31;
-    const int warp = tid >> 5;
     const int64_t tiles = (a.rows + a.tile_rows - 1) / a.tile_rows;
     const int64_t my_tiles = tiles > blockIdx.x ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int lse_base = a.tile_rows * a.data_w;  // LSE words follow the rows in a stage
-    const int chunks = a.data_w >> 2;
+    const int tile_rows = a.tile_rows;
+    const int data_w = a.data_w;
+    const int pitch = a.row_pitch_w;
+    const int stage_w = a.stage_w;
+    const int lse_base = tile_rows * data_w;  // LSE words follow the rows in a stage
+    const int chunks = data_w >> 2;
+    const uint32_t pitch_magic = a.pitch_magic;
+    const uint32_t *__restrict__ src = a.src;
+    const uint32_t *__restrict__ lse = a.lse;
 
-    // copies of this CTA's k-th tile into stage k % kPackStages
+    auto tile_rows_of = [&](int64_t k) -> int {
+        const int64_t i0 = (blockIdx.x + k * gridDim.x) * tile_rows;
+        return (int)min((int64_t)tile_rows, a.rows - i0);
+    };
+    // row table of this CTA's k-th tile, into slot k % kPackStages: rows are
+    // ordered [rank][token][head], row (rank, b, h) holds cp_attn_out[b, rank*Hr + h]
+    auto fill_table = [&](int64_t k) {
+        const int64_t i0 = (blockIdx.x + k * gridDim.x) * tile_rows;
+        const int nrows = tile_rows_of(k);
+        const int slot = (int)(k % kPackStages);
+        for (int r = tid; r < nrows; r += kPackThreads) {
+            const uint64_t i = (uint64_t)(i0 + r);
+            const uint64_t rank = div_magic(i, a.per_rank_magic);
+            const uint64_t rem = i - rank * (uint64_t)(a.B * a.Hr);
+            const uint64_t b = div_magic(rem, a.hr_magic);
+            const uint64_t head = rank * (uint64_t)a.Hr + (rem - b * (uint64_t)a.Hr);
+            s_row_src[slot][r] = (int64_t)b * a.src_stride_b_w + (int64_t)head * a.src_stride_h_w;
+            s_row_lse[slot][r] = (int64_t)b * a.lse_stride_b + (int64_t)head;
+        }
+    };
+    // copies of this CTA's k-th tile into stage k % kPackStages: lpr lanes per
+    // source row, consecutive lanes on consecutive 16-byte chunks
+    const int lpr = a.lanes_per_row;
+    const int rpw = 32 / lpr;  // rows per warp at a time
+    const int lane = tid & 31;
+    const int sub = lane % lpr;
+    const int row_first = (tid >> 5) * rpw + lane / lpr;
     auto issue = [&](int64_t k) {
-        const int64_t tile = blockIdx.x + k * gridDim.x;
-        const int64_t i0 = tile * a.tile_rows;
-        const int nrows = (int)min((int64_t)a.tile_rows, a.rows - i0);
-        uint32_t *stage = s_stage + (int)(k % kPackStages) * a.stage_w;
-        // warp w copies rows [r0, r1) of the tile, 32 / lpr rows at a time
-        const int r0 = (nrows * warp) / kWarps;
-        const int r1 = (nrows * (warp + 1)) / kWarps;
-        const int lpr = a.lanes_per_row;
-        const int rpi = 32 / lpr;
-        const int sub = lane % lpr;
-        int r = r0 + lane / lpr;
-        if (r >= r1) return;
-        int64_t rank, b, h;
-        pack_row_coords(i0 + r, a.B, a.Hr, rank, b, h);
-        for (;;) {
-            const int64_t head = rank * a.Hr + h;
-            const uint32_t *src = a.src + b * a.src_stride_b_w + head * a.src_stride_h_w;
-            uint32_t *srow = stage + r * a.data_w;
-            for (int c = sub; c < chunks; c += lpr) cp_async_chunk(srow + 4 * c, src + 4 * c);
-            if (sub == 0) cp_async_word(stage + lse_base + r, a.lse + b * a.lse_stride_b + head);
-            r += rpi;
-            if (r >= r1) break;
-            h += rpi;
-            while (h >= a.Hr) {
-                h -= a.Hr;
-                if (++b == a.B) {
-                    b = 0;
-                    ++rank;
-                }
-            }
+        const int nrows = tile_rows_of(k);
+        const int slot = (int)(k % kPackStages);
+        uint32_t *stage = s_stage + slot * stage_w;
+        for (int r = row_first; r < nrows; r += kPackThreads / lpr) {
+            const uint32_t *srow = src + s_row_src[slot][r];
+            uint32_t *drow = stage + r * data_w;
+            for (int c = sub; c < chunks; c += lpr) cp_async_chunk(drow + 4 * c, srow + 4 * c);
+            if (sub == 0) cp_async_word(stage + lse_base + r, lse + s_row_lse[slot][r]);
         }
     };
 
+    for (int64_t k = 0; k < kPackStages && k < my_tiles; ++k) fill_table(k);
+    __syncthreads();
 #pragma unroll
     for (int k = 0; k < kPackStages - 1; ++k) {
         if (k < my_tiles) issue(k);
         cp_async_commit();
     }
+    __syncthreads();  // every thread is done reading the table slots of tiles 0 .. kPackStages-2
     for (int64_t k = 0; k < my_tiles; ++k) {
         if (k + kPackStages - 1 < my_tiles) issue(k + kPackStages - 1);
         cp_async_commit();
+        // tile k's table slot was last read when tile k's copies were issued: fill it
+        // for tile k + kPackStages while the copies are in flight
+        if (k + kPackStages < my_tiles) fill_table(k + kPackStages);
         cp_async_wait<kPackStages - 1>();  // this thread's copies of tile k have landed
-        __syncthreads();                   // ... and everyone else's
+        __syncthreads();                   // ... and everyone else's (and the table)
 
-        const int64_t tile = blockIdx.x + k * gridDim.x;
-        const int64_t i0 = tile * a.tile_rows;
-        const int nrows = (int)min((int64_t)a.tile_rows, a.rows - i0);
-        const int64_t d0 = i0 * a.row_pitch_w;  // first send word of the tile
-        const int len = nrows * a.row_pitch_w;
-        const uint32_t *stage = s_stage + (int)(k % kPackStages) * a.stage_w;
+        const int64_t i0 = (blockIdx.x + k * gridDim.x) * tile_rows;
+        const int nrows = tile_rows_of(k);
+        const int64_t d0 = i0 * pitch;  // first send word of the tile
+        const int len = nrows * pitch;
+        const uint32_t *stage = s_stage + (int)(k % kPackStages) * stage_w;
         const uint4 *stage_v4 = reinterpret_cast<const uint4 *>(stage);
         auto word_of = [&](int r, int kk) -> uint32_t {  // word kk of packed row r of the tile
-            return kk < a.data_w ? stage[r * a.data_w + kk] : stage[lse_base + r];
+            return kk < data_w ? stage[r * data_w + kk] : stage[lse_base + r];
         };
         const int lead = (int)((4 - (d0 & 3)) & 3);  // words before the first 16-byte boundary
         const int full = (len - lead) >> 2;           // whole 16-byte chunks of the range
@@ -568,9 +580,9 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a) {
         // pass 1: chunks inside one row's data
         for (int g = tid; g < full; g += kPackThreads) {
             const int t0 = lead + 4 * g;
-            const int r = (int)__umulhi((uint32_t)t0, a.pitch_magic);
-            const int kk = t0 - r * a.row_pitch_w;
-            if (kk + 3 < a.data_w) {
+            const int r = (int)__umulhi((uint32_t)t0, pitch_magic);
+            const int kk = t0 - r * pitch;
+            if (kk + 3 < data_w) {
                 const int base = t0 - r;  // stage word of packed word t0
                 const uint4 lo4 = stage_v4[base >> 2];
                 const uint4 hi4 = stage_v4[(base >> 2) + 1];
@@ -582,23 +594,23 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a) {
         }
         // pass 2: the chunk holding each row's LSE word
         for (int r = tid; r < nrows; r += kPackThreads) {
-            const int t_row = r * a.row_pitch_w;
-            const int t_lse = t_row + a.data_w;
+            const int t_row = r * pitch;
+            const int t_lse = t_row + data_w;
             const int g = (t_lse - lead) >> 2;
             if (t_lse >= lead && g < full) {
                 Words<4> o;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int kk = lead + 4 * g + e - t_row;
-                    o.w[e] = kk < a.row_pitch_w ? word_of(r, kk) : word_of(r + 1, kk - a.row_pitch_w);
+                    o.w[e] = kk < pitch ? word_of(r, kk) : word_of(r + 1, kk - pitch);
                 }
                 store_words<4>(dst_full + 4 * g, o);
             }
         }
         // the partial chunks at the two ends of the range (a range has >= 5 words)
         auto word_at = [&](int t) -> uint32_t {
-            const int r = (int)__umulhi((uint32_t)t, a.pitch_magic);
-            return word_of(r, t - r * a.row_pitch_w);
+            const int r = (int)__umulhi((uint32_t)t, pitch_magic);
+            return word_of(r, t - r * pitch);
         };
         if (tid < lead) {
             Words<1> o;
