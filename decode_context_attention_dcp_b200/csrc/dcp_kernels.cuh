@@ -392,41 +392,30 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
                 }
             }
             if constexpr (PACKED && UNIFORM) {
-                // sum c+1 for output chunk c: the next lane's slot k, lane 0's slot k+1 for
-                // lane G-1, the tail sum for the row's last chunk
+                // Round the aligned sums to output words first (rounding is per element,
+                // so it commutes with a whole-word shift), then funnel by q words: output
+                // chunk c = words q.. of sums c and c+1; sum c+1 comes from the next lane
+                // (lane 0's next slot for lane G-1, the tail sum for the row's last chunk).
                 const int q = qv[0];  // the same for every shard
+                Words<4> enc[CPL];
+#pragma unroll
+                for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) enc[k].w[e] = T::encode(&acc[k][e * T::kPerWord]);
+                Words<4> tenc;
+#pragma unroll
+                for (int e = 0; e < 3; ++e) tenc.w[e] = T::encode(&tacc[e * T::kPerWord]);
+                tenc.w[3] = 0u;
 #pragma unroll
                 for (int k = 0; k < CPL; ++k) {
-                    float nx[kElems];
+                    Words<4> send = enc[k];
+                    if (k + 1 < CPL && j == 0) send = enc[k + 1 < CPL ? k + 1 : k];
+                    Words<4> nx;
 #pragma unroll
-                    for (int e = 0; e < 3 * T::kPerWord; ++e) {
-                        const float send = (k + 1 < CPL && j == 0) ? acc[k + 1 < CPL ? k + 1 : k][e] : acc[k][e];
-                        nx[e] = __shfl_sync(0xffffffffu, send, next_lane);
-                    }
-                    if (act[k] && c[k] == a.chunks - 1) {
-#pragma unroll
-                        for (int e = 0; e < 3 * T::kPerWord; ++e) nx[e] = tacc[e];
-                    }
-                    if (act[k]) {
-                        // elements from word q of sum c, then the first words of sum c+1
-                        float outv[kElems];
-#pragma unroll
-                        for (int e = 0; e < kElems; ++e) {
-                            float v = 0.0f;
-#pragma unroll
-                            for (int qq = 0; qq < 4; ++qq) {
-                                const int s2 = e + qq * T::kPerWord;
-                                const float cand = s2 < kElems ? acc[k][s2 < kElems ? s2 : 0]
-                                                               : nx[s2 - kElems < 3 * T::kPerWord ? s2 - kElems : 0];
-                                if (qq == q) v = cand;
-                            }
-                            outv[e] = v;
-                        }
-                        Words<4> o;
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) o.w[e] = T::encode(&outv[e * T::kPerWord]);
-                        store_words<4>(a.result + u * a.data_w + 4 * (int64_t)c[k], o);
-                    }
+                    for (int e = 0; e < 3; ++e) nx.w[e] = __shfl_sync(0xffffffffu, send.w[e], next_lane);
+                    nx.w[3] = 0u;
+                    if (act[k] && c[k] == a.chunks - 1) nx = tenc;
+                    if (act[k]) store_words<4>(a.result + u * a.data_w + 4 * (int64_t)c[k], funnel_words(enc[k], nx, q));
                 }
             } else {
 #pragma unroll
