@@ -85,7 +85,7 @@ bool pack_smem_reserved() {
     if (dev < 64 && done[dev].load(std::memory_order_acquire)) return true;
     const int max_stage_w = (int)(((kMaxD + 1 + 3) & ~int64_t(3)) + 4);  // one fp32 row of kMaxD words
     const size_t bytes = (size_t)dcp::kPackStages * max_stage_w * 4;
-    if (cudaFuncSetAttribute(dcp::pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+    if (cudaFuncSetAttribute(dcp::pack_kernel<>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
         cudaSuccess)
         return false;
     if (dev < 64) done[dev].store(1, std::memory_order_release);
@@ -97,7 +97,7 @@ int pack_resident_ctas(size_t smem) {
     static std::atomic<uint64_t> cache{0};  // (smem << 16) | ctas
     const uint64_t c = cache.load(std::memory_order_relaxed);
     if (c && (c >> 16) == smem) return (int)(c & 0xffff);
-    const int n = resident_ctas(dcp::pack_kernel, dcp::kPackThreads, smem);
+    const int n = resident_ctas(dcp::pack_kernel<>, dcp::kPackThreads, smem);
     cache.store(((uint64_t)smem << 16) | (uint64_t)n, std::memory_order_relaxed);
     return n;
 }
@@ -381,7 +381,7 @@ int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_b
     const int64_t tiles = (a.rows + a.tile_rows - 1) / a.tile_rows;
     const int64_t cap = (int64_t)sm_count() * per_sm;
     const int grid = (int)(tiles < cap ? tiles : cap);
-    dcp::pack_kernel<<<grid, dcp::kPackThreads, smem, static_cast<cudaStream_t>(cuda_stream)>>>(a);
+    dcp::pack_kernel<><<<grid, dcp::kPackThreads, smem, static_cast<cudaStream_t>(cuda_stream)>>>(a);
     return launch_status(fn);
 }
 

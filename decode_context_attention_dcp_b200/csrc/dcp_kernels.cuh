@@ -435,8 +435,8 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
 
 // ---------------------------------------------------------------------------
 // pack
-constexpr int kPackStages = 4;            // shared-memory tiles in flight per CTA
-constexpr int kPackMinStageWords = 4096;  // 16 KiB per tile (more when one row needs it)
+constexpr int kPackStages = 3;            // shared-memory tiles in flight per CTA
+constexpr int kPackMinStageWords = 8192;  // up to 32 KiB per tile (more when one row needs it)
 constexpr int kPackMaxTileRows = 64;      // rows per tile (row tables in shared memory)
 
 struct PackArgs {
@@ -479,7 +479,10 @@ __device__ __forceinline__ uint64_t div_magic(uint64_t n, uint64_t magic) {
 //   the row's LSE word (rows are >= 5 words, so a chunk holds at most one LSE).
 //   The partial chunks at the two ends of the range use 4-byte stores.
 // Every word of the send buffer is written once, by one CTA.
-__global__ void __launch_bounds__(kPackThreads) pack_kernel(const PackArgs a) {
+template <int STAGES = kPackStages, int THREADS = kPackThreads>
+__global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
+    constexpr int kPackStages = STAGES;
+    constexpr int kPackThreads = THREADS;
     extern __shared__ uint4 s_stage_v4[];
     uint32_t *s_stage = reinterpret_cast<uint32_t *>(s_stage_v4);
     __shared__ int64_t s_row_src[kPackStages][kPackMaxTileRows];  // word offset of each source row
