@@ -288,6 +288,13 @@ def run_sweep(args) -> int:
                                             return_lse=w.return_lse)),
             ("dcp_pack", w.pack_bytes(), lambda: dcp.dcp_pack(cp_out, cp_lse, send, w.N)),
         ]
+        if w.B >= 4096 or w is wl.MLA:
+            # the same shards received head-scattered, [N, Hr, B, D] (dcp_lse_combine_strided)
+            hm_out = d_out.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+            hm_lse = d_lse.permute(0, 2, 1).contiguous().permute(0, 2, 1)
+            kernels.append(("dcp_lse_combine_strided[head-major]", w.combine_bytes(),
+                            lambda: dcp.dcp_lse_combine(hm_out, hm_lse, res, gl, is_lse_base_on_e=w.is_lse_base_on_e,
+                                                        return_lse=w.return_lse)))
         for name, nbytes, fn in kernels:
             for _ in range(3):
                 fn()
@@ -306,7 +313,7 @@ def run_sweep(args) -> int:
             gbs = nbytes / (t * 1e-3) / 1e9
             print(f"| {w.name} | {w.N} | {w.B} | {w.Hr} | {w.D} | {w.dtype} | {name} | {nbytes} | {t * 1e3:.1f} | "
                   f"{gbs:.0f} | {gbs / peak:.3f} |", flush=True)
-        del d_out, d_lse, recv, cp_out, cp_lse, res, gl, send
+        del d_out, d_lse, recv, cp_out, cp_lse, res, gl, send, kernels
         torch.cuda.empty_cache()
     return 0
 

@@ -16,6 +16,7 @@ Low-level calls (same names as the C ABI, caller-allocated outputs):
 
 Allocating helpers with the pages' argument conventions:
     lse_weighted_combine(outputs, lses, return_lse=False, is_lse_base_on_e=True)
+    merge_dcp_outputs(output_recv, lse_recv, token_dim)   (head- or token-scattered layouts)
     pack(cp_attn_out, cp_attn_lse, world_size)
     unpack_combine(recv_buf, return_lse=False, is_lse_base_on_e=True)
 """
@@ -30,7 +31,8 @@ from . import _build
 
 __all__ = [
     "DCPError", "library", "dcp_lse_pack_dim", "dcp_pack", "dcp_lse_combine", "dcp_unpack_combine",
-    "dcp_last_error", "dcp_version", "lse_weighted_combine", "pack", "unpack_combine", "DTYPE_CODES",
+    "dcp_last_error", "dcp_version", "lse_weighted_combine", "merge_dcp_outputs", "pack", "unpack_combine",
+    "DTYPE_CODES",
 ]
 
 DTYPE_CODES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
@@ -65,6 +67,10 @@ def library() -> ctypes.CDLL:
                 lib.dcp_lse_combine.argtypes = [_ptr, _ptr, _ptr, _ptr, _i32, _i64, _i64, _i64, _i64, _i64, _i32,
                                                 _i32, _i32, _ptr]
                 lib.dcp_lse_combine.restype = _i32
+                lib.dcp_lse_combine_strided.argtypes = [_ptr, _ptr, _ptr, _ptr, _i32, _i64, _i64, _i64,
+                                                        _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64,
+                                                        _i32, _i32, _i32, _ptr]
+                lib.dcp_lse_combine_strided.restype = _i32
                 lib.dcp_unpack_combine.argtypes = [_ptr, _ptr, _ptr, _i32, _i64, _i64, _i64, _i64, _i32, _i32, _i32,
                                                    _ptr]
                 lib.dcp_unpack_combine.restype = _i32
@@ -155,24 +161,35 @@ def dcp_lse_combine(outputs: torch.Tensor, lses: torch.Tensor, result: torch.Ten
                     return_lse: bool = False, stream=None) -> None:
     """outputs [N, B, H, D] + lses [N, B, H] fp32 -> result [B, H, D] (+ global_lse [B, H] fp32).
 
-    dim 0 of outputs / lses may have any stride (a capacity-strided receive buffer); the rest
-    must be contiguous."""
+    Any strides are accepted (views in token- or head-major order, capacity-strided shards) as
+    long as the last dimension of outputs and result is contiguous: the canonical layout goes to
+    dcp_lse_combine, every other one to dcp_lse_combine_strided."""
     dev = _cuda(outputs, lses, result, global_lse)
     N, B, H, D = outputs.shape
     if lses.shape != (N, B, H) or lses.dtype != torch.float32:
         raise ValueError(f"lses must be fp32 [{N}, {B}, {H}], got {lses.dtype} {tuple(lses.shape)}")
-    _inner_contiguous(outputs, 3, "outputs")
-    _inner_contiguous(lses, 2, "lses")
-    if result.shape != (B, H, D) or result.dtype != outputs.dtype or not result.is_contiguous():
-        raise ValueError("result must be a contiguous [B, H, D] tensor of the output dtype")
-    if return_lse and (global_lse is None or global_lse.shape != (B, H) or global_lse.dtype != torch.float32
-                       or not global_lse.is_contiguous()):
-        raise ValueError("return_lse needs a contiguous fp32 [B, H] global_lse")
+    if outputs.stride(3) != 1 and D > 1:
+        raise ValueError("outputs must be contiguous in its last dimension")
+    if result.shape != (B, H, D) or result.dtype != outputs.dtype or (result.stride(2) != 1 and D > 1):
+        raise ValueError("result must be a [B, H, D] tensor of the output dtype, contiguous in its last dimension")
+    if return_lse and (global_lse is None or global_lse.shape != (B, H) or global_lse.dtype != torch.float32):
+        raise ValueError("return_lse needs an fp32 [B, H] global_lse")
+    gs = global_lse.stride() if (return_lse and global_lse is not None) else (0, 0)
+    canonical = (outputs.stride()[1:] == (H * D, D, 1) or B * H == 1) and lses.stride()[1:] == (H, 1) \
+        and result.is_contiguous() and (not return_lse or global_lse.is_contiguous())
+    if canonical:
+        with torch.cuda.device(dev):
+            _check(library().dcp_lse_combine(
+                outputs.data_ptr(), lses.data_ptr(), result.data_ptr(),
+                global_lse.data_ptr() if (return_lse and global_lse is not None) else None,
+                N, B, H, D, outputs.stride(0) if N > 1 else B * H * D, lses.stride(0) if N > 1 else B * H,
+                _code(outputs.dtype), int(bool(is_lse_base_on_e)), int(bool(return_lse)), _stream(dev, stream)))
+        return
     with torch.cuda.device(dev):
-        _check(library().dcp_lse_combine(
+        _check(library().dcp_lse_combine_strided(
             outputs.data_ptr(), lses.data_ptr(), result.data_ptr(),
             global_lse.data_ptr() if (return_lse and global_lse is not None) else None,
-            N, B, H, D, outputs.stride(0) if N > 1 else B * H * D, lses.stride(0) if N > 1 else B * H,
+            N, B, H, D, *outputs.stride()[:3], *lses.stride(), *result.stride()[:2], gs[0], gs[1],
             _code(outputs.dtype), int(bool(is_lse_base_on_e)), int(bool(return_lse)), _stream(dev, stream)))
 
 
@@ -207,6 +224,24 @@ def lse_weighted_combine(outputs: torch.Tensor, lses: torch.Tensor, return_lse: 
     glse = torch.empty((B, H), dtype=torch.float32, device=outputs.device) if return_lse else None
     dcp_lse_combine(outputs, lses, result, glse, is_lse_base_on_e=is_lse_base_on_e, return_lse=return_lse)
     return (result, glse) if return_lse else result
+
+
+def merge_dcp_outputs(output_recv: torch.Tensor, lse_recv: torch.Tensor, token_dim: int,
+                      return_lse: bool = False, is_lse_base_on_e: bool = True):
+    """The merge of received shards in the layouts of vllm-ascend sfa_cp.py
+    _merge_dcp_outputs_with_torch: output_recv [N, X, Y, D], lse_recv [N, X, Y] fp32, with the
+    tokens on dim ``token_dim`` (1: [N, T, H, D], tokens scattered; 2: [N, H, T, D], heads
+    scattered).  Returns the combine as a contiguous [T, H, D] tensor of the output dtype (and
+    the global LSE [T, H] fp32)."""
+    if token_dim not in (1, 2):
+        raise ValueError(f"token_dim must be 1 or 2, got {token_dim}")
+    if output_recv.dim() != 4 or lse_recv.dim() != 3 or tuple(output_recv.shape[:3]) != tuple(lse_recv.shape):
+        raise ValueError(f"expected [N, X, Y, D] outputs and [N, X, Y] LSEs, got {tuple(output_recv.shape)} and "
+                         f"{tuple(lse_recv.shape)}")
+    if token_dim == 2:
+        output_recv = output_recv.transpose(1, 2)
+        lse_recv = lse_recv.transpose(1, 2)
+    return lse_weighted_combine(output_recv, lse_recv, return_lse=return_lse, is_lse_base_on_e=is_lse_base_on_e)
 
 
 def pack(cp_attn_out: torch.Tensor, cp_attn_lse: torch.Tensor, world_size: int) -> torch.Tensor:

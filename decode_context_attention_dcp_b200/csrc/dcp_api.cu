@@ -245,22 +245,23 @@ int32_t dcp_lse_pack_dim(int32_t dtype) {
     return es ? 4 / es : -1;
 }
 
-int32_t dcp_lse_combine(const void *outputs, const float *lses, void *result, float *global_lse, int32_t N, int64_t B,
-                        int64_t H, int64_t D, int64_t out_stride_n, int64_t lse_stride_n, int32_t dtype,
-                        int32_t is_lse_base_on_e, int32_t return_lse, void *cuda_stream) {
-    const char *fn = "dcp_lse_combine";
+namespace {
+
+// The split-layout combine with every stride explicit (elements of each array).
+int32_t lse_combine_impl(const char *fn, const void *outputs, const float *lses, void *result, float *global_lse,
+                         int32_t N, int64_t B, int64_t H, int64_t D, int64_t os_n, int64_t os_b, int64_t os_h,
+                         int64_t ls_n, int64_t ls_b, int64_t ls_h, int64_t rs_b, int64_t rs_h, int64_t gs_b,
+                         int64_t gs_h, int32_t dtype, int32_t is_lse_base_on_e, int32_t return_lse,
+                         void *cuda_stream) {
     int32_t st = check_common(fn, dtype, N, B, H, D);
     if (st != DCP_OK) return st;
     const int es = elem_size(dtype);
-    if (out_stride_n < B * H * D)
-        return fail(DCP_ERR_INVALID_ARG, "%s: out_stride_n %lld < B*H*D = %lld", fn, (long long)out_stride_n,
-                    (long long)(B * H * D));
-    if (lse_stride_n < B * H)
-        return fail(DCP_ERR_INVALID_ARG, "%s: lse_stride_n %lld < B*H = %lld", fn, (long long)lse_stride_n,
-                    (long long)(B * H));
-    if ((out_stride_n * es) % 16 != 0)
-        return fail(DCP_ERR_MISALIGNED, "%s: out_stride_n %lld elements is not a multiple of 16 bytes", fn,
-                    (long long)out_stride_n);
+    const int64_t vec = 16 / es;  // elements per 16 bytes
+    if (os_n < 0 || os_b < 0 || os_h < 0 || ls_n < 0 || ls_b < 0 || ls_h < 0 || rs_b < 0 || rs_h < 0 || gs_b < 0 ||
+        gs_h < 0)
+        return fail(DCP_ERR_INVALID_ARG, "%s: negative stride", fn);
+    if (os_n % vec || os_b % vec || os_h % vec || rs_b % vec || rs_h % vec)
+        return fail(DCP_ERR_MISALIGNED, "%s: output and result strides must be multiples of 16 bytes", fn);
     if (B == 0) return ok();
     if (!outputs || !lses || !result) return fail(DCP_ERR_INVALID_ARG, "%s: null buffer pointer", fn);
     if (return_lse && !global_lse) return fail(DCP_ERR_INVALID_ARG, "%s: return_lse set but global_lse is null", fn);
@@ -268,6 +269,7 @@ int32_t dcp_lse_combine(const void *outputs, const float *lses, void *result, fl
         return fail(DCP_ERR_MISALIGNED, "%s: outputs and result must be 16-byte aligned", fn);
     if (!aligned(lses, 4) || (return_lse && !aligned(global_lse, 4)))
         return fail(DCP_ERR_MISALIGNED, "%s: lses and global_lse must be 4-byte aligned", fn);
+    if (B * H >= (int64_t(1) << 32)) return fail(DCP_ERR_INVALID_ARG, "%s: more than 2^32 result rows", fn);
 
     dcp::CombineArgs a{};
     a.src = static_cast<const uint32_t *>(outputs);
@@ -275,15 +277,58 @@ int32_t dcp_lse_combine(const void *outputs, const float *lses, void *result, fl
     a.result = static_cast<uint32_t *>(result);
     a.glse = global_lse;
     a.units = B * H;
-    a.shard_stride_w = out_stride_n * es / 4;
-    a.lse_stride_n = lse_stride_n;
+    a.shard_stride_w = os_n * es / 4;
+    a.lse_stride_n = ls_n;
     a.data_w = (int32_t)(D * es / 4);
     a.row_pitch_w = a.data_w;
     a.chunks = a.data_w / 4;
+    a.heads = H;
+    a.heads_magic = magic64((uint64_t)H);
+    a.src_sb_w = os_b * es / 4;
+    a.src_sh_w = os_h * es / 4;
+    a.lse_sb = ls_b;
+    a.lse_sh = ls_h;
+    a.res_sb_w = rs_b * es / 4;
+    a.res_sh_w = rs_h * es / 4;
+    a.glse_sb = gs_b;
+    a.glse_sh = gs_h;
     a.N = N;
     a.base_e = is_lse_base_on_e ? 1 : 0;
     a.return_lse = return_lse ? 1 : 0;
     return dispatch_dtype<false>(dtype, a, static_cast<cudaStream_t>(cuda_stream));
+}
+
+}  // namespace
+
+int32_t dcp_lse_combine(const void *outputs, const float *lses, void *result, float *global_lse, int32_t N, int64_t B,
+                        int64_t H, int64_t D, int64_t out_stride_n, int64_t lse_stride_n, int32_t dtype,
+                        int32_t is_lse_base_on_e, int32_t return_lse, void *cuda_stream) {
+    const char *fn = "dcp_lse_combine";
+    int32_t st = check_common(fn, dtype, N, B, H, D);
+    if (st != DCP_OK) return st;
+    if (out_stride_n < B * H * D)
+        return fail(DCP_ERR_INVALID_ARG, "%s: out_stride_n %lld < B*H*D = %lld", fn, (long long)out_stride_n,
+                    (long long)(B * H * D));
+    if (lse_stride_n < B * H)
+        return fail(DCP_ERR_INVALID_ARG, "%s: lse_stride_n %lld < B*H = %lld", fn, (long long)lse_stride_n,
+                    (long long)(B * H));
+    if ((out_stride_n * elem_size(dtype)) % 16 != 0)
+        return fail(DCP_ERR_MISALIGNED, "%s: out_stride_n %lld elements is not a multiple of 16 bytes", fn,
+                    (long long)out_stride_n);
+    return lse_combine_impl(fn, outputs, lses, result, global_lse, N, B, H, D, out_stride_n, H * D, D, lse_stride_n,
+                            H, 1, H * D, D, H, 1, dtype, is_lse_base_on_e, return_lse, cuda_stream);
+}
+
+int32_t dcp_lse_combine_strided(const void *outputs, const float *lses, void *result, float *global_lse, int32_t N,
+                                int64_t B, int64_t H, int64_t D, int64_t out_stride_n, int64_t out_stride_b,
+                                int64_t out_stride_h, int64_t lse_stride_n, int64_t lse_stride_b,
+                                int64_t lse_stride_h, int64_t result_stride_b, int64_t result_stride_h,
+                                int64_t glse_stride_b, int64_t glse_stride_h, int32_t dtype, int32_t is_lse_base_on_e,
+                                int32_t return_lse, void *cuda_stream) {
+    return lse_combine_impl("dcp_lse_combine_strided", outputs, lses, result, global_lse, N, B, H, D, out_stride_n,
+                            out_stride_b, out_stride_h, lse_stride_n, lse_stride_b, lse_stride_h, result_stride_b,
+                            result_stride_h, glse_stride_b, glse_stride_h, dtype, is_lse_base_on_e, return_lse,
+                            cuda_stream);
 }
 
 int32_t dcp_unpack_combine(const void *recv_buf, void *result, float *global_lse, int32_t N, int64_t B, int64_t Hr,

@@ -135,6 +135,11 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(PENDING) : "memory");
 }
 
+// n / d for n < 2^32 and d <= 2^32, with magic = ceil(2^64 / d) (0 meaning d == 1).
+__device__ __forceinline__ uint64_t div_magic(uint64_t n, uint64_t magic) {
+    return magic ? __umul64hi(n, magic) : n;
+}
+
 // An LSE that is NaN or +-inf becomes -inf; classified on the exponent bits so
 // the rule holds under any compiler math flags.
 __device__ __forceinline__ float sanitize_lse(uint32_t bits) {
@@ -160,13 +165,23 @@ __device__ __forceinline__ float group_sum(float v) {
 struct CombineArgs {
     const uint32_t *src;     // split: outputs; packed: receive buffer (as words)
     const float *lses;       // split layout only
-    uint32_t *result;        // [units, data_w] words
-    float *glse;             // [units], written when return_lse
+    uint32_t *result;        // result rows (as words)
+    float *glse;             // global LSEs, written when return_lse
     int64_t units;           // rows of the result (B * heads)
     int64_t shard_stride_w;  // words between consecutive shards
     int64_t lse_stride_n;    // split layout: floats between consecutive shards
-    int64_t row_pitch_w;     // words between consecutive rows of one shard
+    int64_t row_pitch_w;     // packed layout: words between consecutive rows of one shard
     int64_t total_w;         // packed layout: words of the buffer that may be read
+    // split layout: row (b, h) of a shard at b*src_sb_w + h*src_sh_w, its LSE at
+    // b*lse_sb + h*lse_sh, the result row at b*res_sb_w + h*res_sh_w and the global
+    // LSE at b*glse_sb + h*glse_sh.  The packed layout's result is [units, data_w]
+    // and its global LSE [units], contiguous.
+    int64_t heads;           // H: unit u is (b, h) = (u / H, u mod H)
+    uint64_t heads_magic;    // ceil(2^64 / H), 0 when H == 1
+    int64_t src_sb_w, src_sh_w;
+    int64_t lse_sb, lse_sh;
+    int64_t res_sb_w, res_sh_w;
+    int64_t glse_sb, glse_sh;
     int32_t data_w;          // words of data per row (D * elemsize / 4), a multiple of 4
     int32_t chunks;          // data_w / 4: 16-byte chunks per row
     int32_t slots;           // ceil(chunks / G): chunk slots per lane
@@ -247,7 +262,20 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
     for (int64_t task = (int64_t)blockIdx.x * kWarps + warp; task < tasks; task += (int64_t)gridDim.x * kWarps) {
         const int64_t u = task * kUnitsPerWarp + ul;
         const bool valid = u < a.units;
-        const int64_t row = u * a.row_pitch_w;
+        int64_t row, lse_off, res_off, glse_off;
+        if constexpr (PACKED) {
+            row = u * a.row_pitch_w;
+            res_off = u * a.data_w;
+            glse_off = u;
+            lse_off = 0;
+        } else {
+            const int64_t b = (int64_t)div_magic((uint64_t)u, a.heads_magic);
+            const int64_t h = u - b * a.heads;
+            row = b * a.src_sb_w + h * a.src_sh_w;
+            lse_off = b * a.lse_sb + h * a.lse_sh;
+            res_off = b * a.res_sb_w + h * a.res_sh_w;
+            glse_off = b * a.glse_sb + h * a.glse_sh;
+        }
 
         int c[CPL];
         bool act[CPL];
@@ -296,7 +324,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
                     const int q = (int)(w0 & 3);
                     bits = q == 0 ? t.w[0] : q == 1 ? t.w[1] : q == 2 ? t.w[2] : t.w[3];
                 } else {
-                    bits = load_word(reinterpret_cast<const uint32_t *>(a.lses) + n * a.lse_stride_n + u);
+                    bits = load_word(reinterpret_cast<const uint32_t *>(a.lses) + n * a.lse_stride_n + lse_off);
                 }
                 l = sanitize_lse(bits);
             }
@@ -316,7 +344,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
         wsum = group_sum<G>(wsum);
         const float denom = fmaxf(wsum, 1e-10f);
         for (int n = j; n < a.N; n += G) sw[n] = sw[n] / denom;
-        if (a.return_lse && valid && j == 0) a.glse[u] = (a.base_e ? logf(wsum) : log2f(wsum)) + m;
+        if (a.return_lse && valid && j == 0) a.glse[glse_off] = (a.base_e ? logf(wsum) : log2f(wsum)) + m;
 
         // UNIFORM: weighted sum of the shards' tail chunks, reduced over the lane group
         float tacc[kElems];
@@ -415,7 +443,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
                     for (int e = 0; e < 3; ++e) nx.w[e] = __shfl_sync(0xffffffffu, send.w[e], next_lane);
                     nx.w[3] = 0u;
                     if (act[k] && c[k] == a.chunks - 1) nx = tenc;
-                    if (act[k]) store_words<4>(a.result + u * a.data_w + 4 * (int64_t)c[k], funnel_words(enc[k], nx, q));
+                    if (act[k]) store_words<4>(a.result + res_off + 4 * (int64_t)c[k], funnel_words(enc[k], nx, q));
                 }
             } else {
 #pragma unroll
@@ -424,7 +452,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
                         Words<4> o;
 #pragma unroll
                         for (int e = 0; e < 4; ++e) o.w[e] = T::encode(&acc[k][e * T::kPerWord]);
-                        store_words<4>(a.result + u * a.data_w + 4 * (int64_t)c[k], o);
+                        store_words<4>(a.result + res_off + 4 * (int64_t)c[k], o);
                     }
                 }
             }
@@ -458,11 +486,6 @@ struct PackArgs {
     int32_t tile_rows;        // packed rows per tile
     int32_t stage_w;          // words per shared-memory stage (a multiple of 4)
 };
-
-// n / d for n < 2^32 and d <= 2^32, with magic = ceil(2^64 / d) (0 meaning d == 1).
-__device__ __forceinline__ uint64_t div_magic(uint64_t n, uint64_t magic) {
-    return magic ? __umul64hi(n, magic) : n;
-}
 
 // A CTA packs tiles of `tile_rows` consecutive packed rows (one contiguous word
 // range of the send buffer), kPackStages tiles in flight.

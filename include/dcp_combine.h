@@ -8,9 +8,10 @@
  * the LSE-weighted combine of the N partials.  This library runs the three
  * device steps of that combine, all inside one GPU's memory:
  *
- *   dcp_pack            partial output + fp32 LSE -> one packed send buffer
- *   dcp_lse_combine     combine of separate output / LSE receive buffers
- *   dcp_unpack_combine  combine read straight out of the packed buffer
+ *   dcp_pack                 partial output + fp32 LSE -> one packed send buffer
+ *   dcp_lse_combine          combine of separate output / LSE receive buffers
+ *   dcp_lse_combine_strided  the same with any token / head layout
+ *   dcp_unpack_combine       combine read straight out of the packed buffer
  *
  * Defining passages (web pages, by title and section):
  *   [COMBINE] vLLM API docs, vllm.v1.attention.ops.dcp_alltoall,
@@ -23,6 +24,9 @@
  *             split receive buffers received_output [N, T_max, H/N, D] and
  *             received_lse [N, T_max, H/N] (fp32), i.e. a shard stride that
  *             may exceed B*H*D.
+ *   [ASCEND]  vllm-ascend, vllm_ascend/attention/context_parallel/sfa_cp.py,
+ *             _merge_dcp_outputs_with_torch: the same merge as a softmax over
+ *             the shard axis, on head- or token-scattered receive layouts.
  *
  * The combine, per token b and head h, over shards n = 0..N-1 ([COMBINE]):
  *   l_n <- -inf if l_n is NaN or +-inf
@@ -58,7 +62,7 @@ extern "C" {
 #endif
 
 /* Element type of the attention outputs and of the packed buffer.  LSEs are
- * always fp32 ([A2A]: "cp_attn_lse: [B, H] log-sum-exp values (fp32)"). */
+ * always fp32, as [A2A] specifies for the partial LSE. */
 typedef enum {
     DCP_BF16 = 0,
     DCP_FP16 = 1,
@@ -129,6 +133,35 @@ int32_t dcp_lse_combine(const void *outputs, const float *lses, void *result, fl
                         int32_t N, int64_t B, int64_t H, int64_t D,
                         int64_t out_stride_n, int64_t lse_stride_n, int32_t dtype,
                         int32_t is_lse_base_on_e, int32_t return_lse, void *cuda_stream);
+
+/*
+ * The same combine with every layout stride explicit: split receive buffers in
+ * any token / head order.  This covers the layouts in which the vllm-ascend
+ * sfa_cp.py merge (_merge_dcp_outputs_with_torch, _merge_dcp_outputs) receives
+ * the shards: head-scattered [N, H/N, T, D] with LSEs [N, H/N, T]
+ * ("token_dim = 2"), and token-scattered [N, T/N, H, D] ("token_dim = 1"),
+ * as well as capacity-strided [DIRECT] buffers.
+ *
+ * outputs     element (n, b, h, d) at n*out_stride_n + b*out_stride_b +
+ *             h*out_stride_h + d.
+ * lses        fp32; element (n, b, h) at n*lse_stride_n + b*lse_stride_b +
+ *             h*lse_stride_h.
+ * result      element (b, h, d) at b*result_stride_b + h*result_stride_h + d.
+ * global_lse  fp32; element (b, h) at b*glse_stride_b + h*glse_stride_h;
+ *             written only when return_lse != 0 (may be NULL otherwise).
+ * Strides are in elements of each array and >= 0; inputs may overlap one
+ * another (they are only read); result rows must not overlap.
+ *
+ * Requirements: as dcp_lse_combine, and out_stride_* and result_stride_*
+ * multiples of 16 bytes (else DCP_ERR_MISALIGNED); B*H < 2^32.
+ */
+int32_t dcp_lse_combine_strided(const void *outputs, const float *lses, void *result, float *global_lse,
+                                int32_t N, int64_t B, int64_t H, int64_t D,
+                                int64_t out_stride_n, int64_t out_stride_b, int64_t out_stride_h,
+                                int64_t lse_stride_n, int64_t lse_stride_b, int64_t lse_stride_h,
+                                int64_t result_stride_b, int64_t result_stride_h,
+                                int64_t glse_stride_b, int64_t glse_stride_h, int32_t dtype,
+                                int32_t is_lse_base_on_e, int32_t return_lse, void *cuda_stream);
 
 /*
  * Fused unpack + combine over the packed receive buffer ([A2A], the step

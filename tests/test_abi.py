@@ -149,3 +149,29 @@ def test_binding_rejects_cpu_tensors():
         dcp.lse_weighted_combine(x, lse)
     with pytest.raises((dcp.DCPError, ValueError)):
         dcp.dcp_lse_pack_dim(torch.int8)
+
+
+def _strided(lib, **kw):
+    a = dict(outputs=A, lses=A, result=A, glse=A, N=2, B=4, H=8, D=128, dtype=0, ret=1)
+    B, H, D = kw.get("B", 4), kw.get("H", 8), kw.get("D", 128)
+    st = dict(os_n=B * H * D, os_b=D, os_h=B * D, ls_n=B * H, ls_b=1, ls_h=B, rs_b=H * D, rs_h=D, gs_b=H, gs_h=1)
+    a.update(st)
+    a.update(kw)
+    return lib.dcp_lse_combine_strided(a["outputs"], a["lses"], a["result"], a["glse"], a["N"], a["B"], a["H"],
+                                       a["D"], a["os_n"], a["os_b"], a["os_h"], a["ls_n"], a["ls_b"], a["ls_h"],
+                                       a["rs_b"], a["rs_h"], a["gs_b"], a["gs_h"], a["dtype"], 1, a["ret"], None)
+
+
+def test_strided_rejections(lib):
+    assert _strided(lib, B=0) == OK
+    assert _strided(lib, dtype=5) == DTYPE
+    assert _strided(lib, N=0) == INVALID
+    assert _strided(lib, os_b=-128) == INVALID
+    assert _strided(lib, ls_h=-1) == INVALID
+    assert _strided(lib, os_b=132) == MISALIGNED          # 264-byte token stride
+    assert _strided(lib, os_n=4 * 8 * 128 + 4) == MISALIGNED
+    assert _strided(lib, rs_h=130) == MISALIGNED
+    assert _strided(lib, result=A + 8) == MISALIGNED
+    assert _strided(lib, glse=None) == INVALID
+    assert _strided(lib, B=1 << 22, H=1 << 10) == INVALID  # 2^32 result rows
+    assert "dcp_lse_combine_strided" in dcp.dcp_last_error()

@@ -347,3 +347,70 @@ def test_errors_raise():
     assert e.value.status == 3
     with pytest.raises(ValueError):
         dcp.pack(torch.zeros((2, 6, 128), dtype=torch.bfloat16, device="cuda"), torch.zeros((2, 6), device="cuda"), 4)
+
+
+# ---- layouts of the received shards (strided combine) -------------------------------------
+@pytest.mark.parametrize("token_dim", [1, 2])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16", "fp32"])
+def test_merge_layouts(o, token_dim, dtype):
+    """The merge layouts of vllm-ascend sfa_cp.py: tokens on dim 1 ([N, T, H, D], tokens scattered)
+    or on dim 2 ([N, H, T, D], heads scattered); the result is [T, H, D] contiguous."""
+    w, outputs, lses = _case(6, 37, 5, 128, dtype, 13)
+    ref_y, ref_g = o.lse_combine(raw(outputs), ORACLE_CODE[outputs.dtype], raw(lses), return_lse=True)
+    if token_dim == 2:
+        recv, lrecv = outputs.permute(0, 2, 1, 3).contiguous(), lses.permute(0, 2, 1).contiguous()
+    else:
+        recv, lrecv = outputs, lses
+    y, g = dcp.merge_dcp_outputs(recv.cuda(), lrecv.cuda(), token_dim, return_lse=True)
+    assert y.is_contiguous() and tuple(y.shape) == (37, 5, 128)
+    assert_out_close(y, ref_y, f"merge token_dim={token_dim}")
+    assert_lse_close(g, ref_g, f"merge token_dim={token_dim} lse")
+
+
+def test_strided_views(o):
+    """Every operand a permuted view of storage in another order."""
+    N, B, H, D = 5, 19, 6, 64
+    w, outputs, lses = _case(N, B, H, D, "bf16", 17)
+    ref_y, ref_g = o.lse_combine(raw(outputs), orc.BF16, raw(lses), return_lse=True)
+    out_store = outputs.permute(1, 2, 0, 3).contiguous().cuda()       # [B, H, N, D]
+    lse_store = lses.permute(2, 0, 1).contiguous().cuda()              # [H, N, B]
+    out_view = out_store.permute(2, 0, 1, 3)                           # [N, B, H, D]
+    lse_view = lse_store.permute(1, 2, 0)                              # [N, B, H]
+    res_store = torch.full((H, B, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gl_store = torch.full((H, B), float("nan"), device="cuda")
+    dcp.dcp_lse_combine(out_view, lse_view, res_store.permute(1, 0, 2), gl_store.t(), return_lse=True)
+    assert_out_close(res_store.permute(1, 0, 2), ref_y, "strided result")
+    assert_lse_close(gl_store.t(), ref_g, "strided global lse")
+
+
+def test_mla_head_scattered_full_size(o):
+    """The MLA workload received head-scattered ([N, Hr, B, D]), element by element."""
+    w = wl.MLA
+    outputs, lses = wl.split_inputs(w)
+    recv = outputs.permute(0, 2, 1, 3).contiguous().cuda()
+    lrecv = lses.permute(0, 2, 1).contiguous().cuda()
+    y, g = dcp.merge_dcp_outputs(recv, lrecv, 2, return_lse=True, is_lse_base_on_e=False)
+    ry, rg = o.lse_combine(raw(outputs), orc.BF16, raw(lses), return_lse=True, is_lse_base_on_e=False)
+    assert_out_close(y, ry, "mla head-scattered")
+    assert_lse_close(g, rg, "mla head-scattered lse")
+
+
+def test_c_entry_points_directly(o):
+    """dcp_lse_combine and dcp_lse_combine_strided called through ctypes with raw pointers agree
+    with the oracle (and with each other) on the same capacity-strided buffers."""
+    lib = dcp.library()
+    N, T_max, B, H, D = 3, 40, 33, 4, 128
+    w, outputs, lses = _case(N, T_max, H, D, "fp16", 23)
+    d_out, d_lse = outputs.cuda(), lses.cuda()
+    ry, rg = o.lse_combine(raw(outputs[:, :B]), orc.FP16, raw(lses[:, :B]), return_lse=True)
+    y1 = torch.empty((B, H, D), dtype=torch.float16, device="cuda")
+    g1 = torch.empty((B, H), device="cuda")
+    y2, g2 = torch.empty_like(y1), torch.empty_like(g1)
+    s = torch.cuda.current_stream().cuda_stream
+    assert lib.dcp_lse_combine(d_out.data_ptr(), d_lse.data_ptr(), y1.data_ptr(), g1.data_ptr(), N, B, H, D,
+                               T_max * H * D, T_max * H, 1, 1, 1, s) == 0
+    assert lib.dcp_lse_combine_strided(d_out.data_ptr(), d_lse.data_ptr(), y2.data_ptr(), g2.data_ptr(), N, B, H, D,
+                                       T_max * H * D, H * D, D, T_max * H, H, 1, H * D, D, H, 1, 1, 1, 1, s) == 0
+    assert_out_close(y1, ry, "dcp_lse_combine")
+    assert_lse_close(g1, rg, "dcp_lse_combine lse")
+    assert torch.equal(y1, y2) and torch.equal(g1, g2)
