@@ -346,12 +346,18 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
         for (int n = j; n < a.N; n += G) sw[n] = sw[n] / denom;
         if (a.return_lse && valid && j == 0) a.glse[glse_off] = (a.base_e ? logf(wsum) : log2f(wsum)) + m;
 
-        // UNIFORM: weighted sum of the shards' tail chunks, reduced over the lane group
+        // UNIFORM: weighted sum of the shards' tail chunks.  With few shards the lane
+        // that owns the row's last chunk sums them itself; otherwise each lane sums its
+        // shards and the group reduces.
         float tacc[kElems];
         if constexpr (PACKED && UNIFORM) {
 #pragma unroll
             for (int e = 0; e < kElems; ++e) tacc[e] = 0.0f;
-            for (int n = j; n < a.N; n += G) {
+            const bool few = a.N <= 4;  // the same for the whole warp
+            const int n_first = few ? 0 : j;
+            const int n_step = few ? 1 : G;
+            const bool owner = j == (a.chunks - 1) % G;
+            for (int n = n_first; n < a.N && (!few || owner); n += n_step) {
                 const uint4 t = s_tail[n];
                 const float w = sw[n];
                 const uint32_t tw[4] = {t.x, t.y, t.z, t.w};
@@ -365,8 +371,10 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
                 }
             }
             // only the first 3 words (the most a row can leave in its tail chunk) matter
+            if (!few) {
 #pragma unroll
-            for (int e = 0; e < 3 * T::kPerWord; ++e) tacc[e] = group_sum<G>(tacc[e]);
+                for (int e = 0; e < 3 * T::kPerWord; ++e) tacc[e] = group_sum<G>(tacc[e]);
+            }
         }
         __syncwarp();
 
