@@ -11,6 +11,9 @@ Sources, by page and section:
     (the combine) and ``dcp_a2a_lse_reduce`` (the packed [N, B, H/N, D+pack] layout).
   * vllm-ascend ``attention/context_parallel/sfa_cp.py``: ``_merge_dcp_outputs_with_torch``
     (the softmax form of the merge) and ``_get_dcp_local_seq_lens`` (interleaved KV shards).
+  * vLLM API docs, ``vllm.v1.attention.ops.dcp``: ``DirectDCPA2AWorkspace.lse_reduce`` takes
+    optional ``seq_lens`` / ``query_start_loc``; what it does with them is not on the pages, so
+    ``lse_combine_varlen`` implements a stated reading (parity unpinned for that reading).
 """
 from __future__ import annotations
 
@@ -80,6 +83,10 @@ class Oracle:
         lib.oracle_attention.argtypes = [_c_ptr, _c_ptr, _c_ptr, _c_int, _c_ptr, _c_ptr, _c_i64, _c_i64,
                                          _c_ptr, _c_i64, ctypes.c_double, _c_int]
         lib.oracle_attention.restype = _c_int
+        lib.oracle_lse_combine_varlen.argtypes = [_c_ptr, _c_int, _c_ptr, _c_int, _c_ptr, _c_ptr, _c_int, _c_i64,
+                                                  _c_i64, _c_i64, _c_i64, _c_i64, _c_ptr, _c_ptr, _c_int, _c_int,
+                                                  _c_int, _c_int]
+        lib.oracle_lse_combine_varlen.restype = _c_int
         lib.oracle_local_seq_len.argtypes = [_c_i64, _c_i64, _c_i64, _c_i64]
         lib.oracle_local_seq_len.restype = _c_i64
         self.lib = lib
@@ -225,6 +232,26 @@ class Oracle:
                                        float(scale), int(is_lse_base_on_e))
         self._check(rc, "attention")
         return out, lse
+
+    def lse_combine_varlen(self, outputs: np.ndarray, out_dtype: int, lses: np.ndarray, seq_lens, query_start_loc,
+                           interleave: int = 1, return_lse: bool = False, is_lse_base_on_e: bool = True):
+        """The combine with empty shards skipped (see oracle_lse_combine_varlen for the reading):
+        outputs [N, T, H, D], lses [N, T, H]; seq_lens [R], query_start_loc [R + 1] (int32)."""
+        outputs = np.ascontiguousarray(outputs)
+        lses = np.ascontiguousarray(lses)
+        N, B, H, D = outputs.shape
+        sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+        qsl = np.ascontiguousarray(np.asarray(query_start_loc, dtype=np.int32))
+        assert qsl.shape[0] == sl.shape[0] + 1
+        lse_dtype = F64 if lses.dtype == np.float64 else FP32
+        result = np.zeros((B, H, D), dtype=np.float64)
+        glse = np.zeros((B, H), dtype=np.float64)
+        rc = self.lib.oracle_lse_combine_varlen(self._ptr(outputs), out_dtype, self._ptr(lses), lse_dtype,
+                                                self._ptr(result), self._ptr(glse), N, B, H, D, B * H * D, B * H,
+                                                self._ptr(sl) if len(sl) else None, self._ptr(qsl), len(sl),
+                                                int(interleave), int(is_lse_base_on_e), int(return_lse))
+        self._check(rc, "lse_combine_varlen")
+        return (result, glse) if return_lse else result
 
     def local_seq_len(self, seq_len: int, cp_size: int, rank: int, interleave: int) -> int:
         return self.lib.oracle_local_seq_len(seq_len, cp_size, rank, interleave)

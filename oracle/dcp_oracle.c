@@ -81,8 +81,9 @@ static double load_elem(const void *base, int dtype, int64_t i) {
 double oracle_decode(const void *base, int dtype, int64_t i) { return load_elem(base, dtype, i); }
 
 /* Number of output-dtype slots that hold one fp32 LSE in a packed row.
- * [A2A] dcp_a2a_lse_reduce packs "the output and fp32 LSE ... into a single
- * output-dtype buffer"; the plainest lossless reading is 4 bytes / itemsize. */
+ * [A2A] dcp_a2a_lse_reduce sends each output row and its fp32 LSE together in
+ * one buffer of the output dtype; the plainest lossless reading is
+ * 4 bytes / itemsize. */
 int oracle_lse_pack_dim(int dtype) {
     if (dtype == ORC_BF16 || dtype == ORC_FP16) return 2;
     if (dtype == ORC_FP32) return 1;
@@ -150,6 +151,51 @@ int oracle_unpack(const void *recv_buf, void *outputs, float *lses,
 }
 
 /*
+ * One (b, h) row of the combine, the [COMBINE] rules in their order.  `empty`
+ * (NULL = none) marks shards whose row holds no context: their LSE counts as
+ * -inf and their output row is never read.  l and w are N-entry scratch.
+ */
+static void combine_row(const void *outputs, int out_dtype, const void *lses, int lse_dtype,
+                        double *result, double *global_lse, int N, int64_t b, int64_t h,
+                        int64_t B, int64_t H, int64_t D, int64_t out_stride_n, int64_t lse_stride_n,
+                        int is_lse_base_on_e, int return_lse, const int *empty,
+                        double *l, double *w) {
+    (void)B; /* rows are addressed (b * H + h); B is the layout's extent */
+    /* step 1: sanitise */
+    for (int n = 0; n < N; ++n) {
+        double v = (empty && empty[n]) ? -INFINITY
+                                       : load_elem(lses, lse_dtype, n * lse_stride_n + b * H + h);
+        l[n] = (isnan(v) || isinf(v)) ? -INFINITY : v;
+    }
+    /* step 2: max over shards, an all -inf max becomes 0 */
+    double m = l[0];
+    for (int n = 1; n < N; ++n)
+        if (l[n] > m) m = l[n];
+    if (m == -INFINITY) m = 0.0;
+    /* step 3: weights */
+    for (int n = 0; n < N; ++n) {
+        w[n] = is_lse_base_on_e ? exp(l[n] - m) : pow(2.0, l[n] - m);
+        if (isnan(w[n])) w[n] = 0.0;
+    }
+    /* step 4: normalise by the clamped sum */
+    double S = 0.0;
+    for (int n = 0; n < N; ++n) S += w[n];
+    double denom = S < 1e-10 ? 1e-10 : S;
+    for (int n = 0; n < N; ++n) w[n] = w[n] / denom;
+    /* step 5: weighted sum over shards */
+    for (int64_t d = 0; d < D; ++d) {
+        double acc = 0.0;
+        for (int n = 0; n < N; ++n)
+            if (!(empty && empty[n]))
+                acc += load_elem(outputs, out_dtype, n * out_stride_n + (b * H + h) * D + d) * w[n];
+        result[(b * H + h) * D + d] = acc;
+    }
+    /* step 6: global LSE from the unclamped sum */
+    if (return_lse)
+        global_lse[b * H + h] = (is_lse_base_on_e ? log(S) : log2(S)) + m;
+}
+
+/*
  * The combine, following [A2A] _lse_weighted_combine step by step, for every
  * token b and head h:
  *   1. an LSE that is NaN or +-inf becomes -inf;
@@ -173,40 +219,10 @@ int oracle_lse_combine(const void *outputs, int out_dtype, const void *lses, int
     double *l = (double *)malloc(sizeof(double) * (size_t)N);
     double *w = (double *)malloc(sizeof(double) * (size_t)N);
     if (!l || !w) { free(l); free(w); return -1; }
-    for (int64_t b = 0; b < B; ++b) {
-        for (int64_t h = 0; h < H; ++h) {
-            /* step 1: sanitise */
-            for (int n = 0; n < N; ++n) {
-                double v = load_elem(lses, lse_dtype, n * lse_stride_n + b * H + h);
-                l[n] = (isnan(v) || isinf(v)) ? -INFINITY : v;
-            }
-            /* step 2: max over shards, an all -inf max becomes 0 */
-            double m = l[0];
-            for (int n = 1; n < N; ++n)
-                if (l[n] > m) m = l[n];
-            if (m == -INFINITY) m = 0.0;
-            /* step 3: weights */
-            for (int n = 0; n < N; ++n) {
-                w[n] = is_lse_base_on_e ? exp(l[n] - m) : pow(2.0, l[n] - m);
-                if (isnan(w[n])) w[n] = 0.0;
-            }
-            /* step 4: normalise by the clamped sum */
-            double S = 0.0;
-            for (int n = 0; n < N; ++n) S += w[n];
-            double denom = S < 1e-10 ? 1e-10 : S;
-            for (int n = 0; n < N; ++n) w[n] = w[n] / denom;
-            /* step 5: weighted sum over shards */
-            for (int64_t d = 0; d < D; ++d) {
-                double acc = 0.0;
-                for (int n = 0; n < N; ++n)
-                    acc += load_elem(outputs, out_dtype, n * out_stride_n + (b * H + h) * D + d) * w[n];
-                result[(b * H + h) * D + d] = acc;
-            }
-            /* step 6: global LSE from the unclamped sum */
-            if (return_lse)
-                global_lse[b * H + h] = (is_lse_base_on_e ? log(S) : log2(S)) + m;
-        }
-    }
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t h = 0; h < H; ++h)
+            combine_row(outputs, out_dtype, lses, lse_dtype, result, global_lse, N, b, h, B, H, D,
+                        out_stride_n, lse_stride_n, is_lse_base_on_e, return_lse, NULL, l, w);
     free(l);
     free(w);
     return 0;
@@ -331,4 +347,46 @@ int64_t oracle_local_seq_len(int64_t seq_len, int64_t cp_size, int64_t rank, int
     if (rem < 0) rem = 0;
     if (rem > interleave) rem = interleave;
     return base + rem;
+}
+
+/*
+ * Variable-length combine: the receive-side reduce of [vLLM API docs,
+ * vllm.v1.attention.ops.dcp, DirectDCPA2AWorkspace.lse_reduce], which takes
+ * optional seq_lens and query_start_loc.  The pages do not say what the op does
+ * with them; the reading taken here (parity of this reading is unpinned):
+ *   - token t belongs to request r when query_start_loc[r] <= t <
+ *     query_start_loc[r + 1] (num_reqs + 1 entries); tokens outside every
+ *     request have no context at all;
+ *   - shard n holds oracle_local_seq_len(seq_lens[r], N, n, interleave) KV
+ *     positions of request r ([ASC] _get_dcp_local_seq_lens); a shard that
+ *     holds none is empty: its LSE counts as -inf and its output row is not
+ *     read (it may never have been written);
+ *   - everything else is oracle_lse_combine.
+ * Same layouts as oracle_lse_combine (split layout, shard strides).
+ */
+int oracle_lse_combine_varlen(const void *outputs, int out_dtype, const void *lses, int lse_dtype,
+                              double *result, double *global_lse, int N, int64_t B, int64_t H, int64_t D,
+                              int64_t out_stride_n, int64_t lse_stride_n, const int32_t *seq_lens,
+                              const int32_t *query_start_loc, int num_reqs, int interleave,
+                              int is_lse_base_on_e, int return_lse) {
+    if (N < 1 || elem_size(out_dtype) == 0 || interleave < 1 || num_reqs < 0) return -1;
+    if (lse_dtype != ORC_FP32 && lse_dtype != ORC_F64) return -1;
+    double *l = (double *)malloc(sizeof(double) * (size_t)N);
+    double *w = (double *)malloc(sizeof(double) * (size_t)N);
+    int *empty = (int *)malloc(sizeof(int) * (size_t)N);
+    if (!l || !w || !empty) { free(l); free(w); free(empty); return -1; }
+    for (int64_t b = 0; b < B; ++b) {
+        int req = -1;
+        for (int r = 0; r < num_reqs; ++r)
+            if (query_start_loc[r] <= b && b < query_start_loc[r + 1]) req = r;
+        for (int n = 0; n < N; ++n)
+            empty[n] = req < 0 || oracle_local_seq_len(seq_lens[req], N, n, interleave) == 0;
+        for (int64_t h = 0; h < H; ++h)
+            combine_row(outputs, out_dtype, lses, lse_dtype, result, global_lse, N, b, h, B, H, D,
+                        out_stride_n, lse_stride_n, is_lse_base_on_e, return_lse, empty, l, w);
+    }
+    free(l);
+    free(w);
+    free(empty);
+    return 0;
 }

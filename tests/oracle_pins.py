@@ -336,3 +336,42 @@ ALL_PINS = [
     pin_local_seq_len,
     pin_bruteforce_attention,
 ]
+
+
+def pin_varlen_reduces_to_combine(o: orc.Oracle) -> None:
+    """The variable-length reading against the plain combine: with every shard holding KV it is the
+    plain combine; an empty shard is the shard's LSE set to -inf with its row never read (NaN
+    there changes nothing); a token outside every request gives 0 and -inf."""
+    rng = np.random.default_rng(13)
+    N, B, H, D = 4, 9, 3, 8
+    raw, code, lses = random_case(rng, N, B, H, D)
+    # three requests: tokens [0,3), [3,7), [7,8); token 8 is padding
+    qsl = [0, 3, 7, 8]
+    for inter in (1, 2):
+        full = [N * inter * 2, 50, 100]
+        y, g = o.lse_combine_varlen(raw, code, lses, full, qsl, inter, return_lse=True)
+        yp, gp = o.lse_combine(raw, code, lses, return_lse=True)
+        np.testing.assert_array_equal(y[:8], yp[:8])
+        np.testing.assert_array_equal(g[:8], gp[:8])
+        assert np.all(y[8] == 0.0) and np.all(g[8] == -np.inf)
+        short = [1, 2 * inter + 1, 0]       # request 0: shard 0 only; request 1: 2-3 shards; request 2: none
+        dirty = raw.copy().view(np.uint16)
+        l2 = lses.copy()
+        for b in range(8):
+            r = 0 if b < 3 else 1 if b < 7 else 2
+            for n in range(N):
+                if o.local_seq_len(short[r], N, n, inter) == 0:
+                    dirty[n, b] = 0x7FC0          # NaN in the rows of empty shards
+                    l2[n, b] = -np.inf
+        yv, gv = o.lse_combine_varlen(dirty, code, lses, short, qsl, inter, return_lse=True)
+        clean = raw.copy()
+        clean[l2 == -np.inf] = 0
+        yr, gr = o.lse_combine(clean, code, l2, return_lse=True)
+        np.testing.assert_allclose(yv[:8], yr[:8], rtol=1e-15, atol=1e-15)
+        assert np.array_equal(np.isinf(gv[:8]), np.isinf(gr[:8]))
+        assert not np.any(np.isnan(yv))
+        assert np.all(yv[8] == 0.0) and np.all(gv[8] == -np.inf)     # padding token
+        assert np.all(yv[7] == 0.0) and np.all(gv[7] == -np.inf)   # request 2 has no KV anywhere
+
+
+ALL_PINS.append(pin_varlen_reduces_to_combine)

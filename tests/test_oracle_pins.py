@@ -67,8 +67,8 @@ MUTANTS = [
      "load_elem(outputs, out_dtype, n * out_stride_n + (b * H + h) * D + d) * w[n];",
      "load_elem(outputs, out_dtype, n * out_stride_n + (h * B + b) * D + d) * w[n];"),
     ("LSE index ignores the shard stride",
-     "load_elem(lses, lse_dtype, n * lse_stride_n + b * H + h);\n                l[n]",
-     "load_elem(lses, lse_dtype, b * H + h);\n                l[n]"),
+     ": load_elem(lses, lse_dtype, n * lse_stride_n + b * H + h);",
+     ": load_elem(lses, lse_dtype, b * H + h);"),
     ("pack sends interleaved heads", "int64_t head = r * Hr + h;", "int64_t head = h * world_size + r;"),
     ("pack puts the LSE first", "memcpy(d + D * es, &cp_attn_lse[b * lse_stride_b + head], 4);",
      "memmove(d + 4, d, (size_t)(D * es - 4)); memcpy(d, &cp_attn_lse[b * lse_stride_b + head], 4);"),
@@ -79,6 +79,10 @@ MUTANTS = [
     ("bf16 decoded from the low bits", "uint32_t w = (uint32_t)bits << 16;", "uint32_t w = (uint32_t)bits;"),
     ("attention LSE misses the max shift", "double lse_e = npos > 0 ? log(z) + mx : -INFINITY;",
      "double lse_e = npos > 0 ? log(z) : -INFINITY;"),
+    ("varlen: empty shard keeps its LSE", "double v = (empty && empty[n]) ? -INFINITY", "double v = 0 ? -INFINITY"),
+    ("varlen: empty shard row still read", "if (!(empty && empty[n]))", "if (1)"),
+    ("varlen: request end inclusive", "query_start_loc[r] <= b && b < query_start_loc[r + 1]",
+     "query_start_loc[r] <= b && b <= query_start_loc[r + 1]"),
     ("local seq len ignores rank", "int64_t rem = seq_len - base * cp_size - rank * interleave;",
      "int64_t rem = seq_len - base * cp_size;"),
 ]
