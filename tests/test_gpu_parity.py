@@ -414,3 +414,38 @@ def test_c_entry_points_directly(o):
     assert_out_close(y1, ry, "dcp_lse_combine")
     assert_lse_close(g1, rg, "dcp_lse_combine lse")
     assert torch.equal(y1, y2) and torch.equal(g1, g2)
+
+
+def test_cuda_graph_replay(o):
+    """pack + unpack+combine captured once in a CUDA graph and replayed on new inputs: the
+    library allocates nothing and never synchronises, so the captured launches stay valid."""
+    N, B, Hr, D = 4, 96, 8, 128
+    H = N * Hr
+    cp_out = torch.empty((B, H, D), dtype=torch.bfloat16, device="cuda")
+    cp_lse = torch.empty((B, H), device="cuda")
+    send = torch.empty((N, B, Hr, D + 2), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((B, Hr, D), dtype=torch.bfloat16, device="cuda")
+    g = torch.empty((B, Hr), device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):  # warm-up (first calls set up per-device state) before capture
+            dcp.dcp_pack(cp_out, cp_lse, send, N)
+            dcp.dcp_unpack_combine(send, y, g, return_lse=True)
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        dcp.dcp_pack(cp_out, cp_lse, send, N)
+        dcp.dcp_unpack_combine(send, y, g, return_lse=True)
+    for seed in (31, 32):
+        w = wl.CombineWorkload("graph", N=N, B=B, Hr=Hr, D=D, lse_lo=-5.0, lse_hi=15.0, p_neginf=0.1, seed=seed)
+        h_out, h_lse = wl.pack_inputs(w)
+        cp_out.copy_(h_out)
+        cp_lse.copy_(h_lse)
+        graph.replay()
+        torch.cuda.synchronize()
+        ref_send = o.pack(raw(h_out), raw(h_lse), N, orc.BF16)
+        assert np.array_equal(bits(send.cpu()), bits(ref_send))
+        ry, rg = o.unpack_combine(ref_send, orc.BF16, D, return_lse=True)
+        assert_out_close(y, ry, f"graph replay seed {seed}")
+        assert_lse_close(g, rg, f"graph replay seed {seed} lse")
