@@ -295,6 +295,17 @@ def run_sweep(args) -> int:
             kernels.append(("dcp_lse_combine_strided[head-major]", w.combine_bytes(),
                             lambda: dcp.dcp_lse_combine(hm_out, hm_lse, res, gl, is_lse_base_on_e=w.is_lse_base_on_e,
                                                         return_lse=w.return_lse)))
+            # a decode batch in which about 30% of the requests are too short to reach every
+            # shard (dcp_lse_combine_varlen reads only the shards that hold KV)
+            seq_lens, qsl = wl.decode_batch(wl.DecodeBatch(B=w.B, p_short=0.3, short_max=w.N, seed=w.seed))
+            req_of = torch.repeat_interleave(torch.arange(len(seq_lens)), qsl[1:] - qsl[:-1])
+            held = torch.clamp(seq_lens.long(), 0, w.N)  # token interleave: min(N, seq) shards hold KV
+            shards_read = int(held[req_of].sum())
+            d_seq, d_qsl = seq_lens.cuda(), qsl.cuda()
+            kernels.append(("dcp_lse_combine_varlen", w.varlen_combine_bytes(shards_read, len(seq_lens)),
+                            lambda: dcp.dcp_lse_combine_varlen(d_out, d_lse, res, d_seq, d_qsl, gl,
+                                                               is_lse_base_on_e=w.is_lse_base_on_e,
+                                                               return_lse=w.return_lse)))
         for name, nbytes, fn in kernels:
             for _ in range(3):
                 fn()

@@ -11,12 +11,14 @@ cannot be built or loaded, every call raises.
 Low-level calls (same names as the C ABI, caller-allocated outputs):
     dcp_pack(cp_attn_out, cp_attn_lse, send_buf, world_size)
     dcp_lse_combine(outputs, lses, result, global_lse=None, ...)
+    dcp_lse_combine_varlen(outputs, lses, result, seq_lens, query_start_loc, ...)
     dcp_unpack_combine(recv_buf, result, global_lse=None, ...)
     dcp_lse_pack_dim(dtype), dcp_last_error()
 
 Allocating helpers with the pages' argument conventions:
     lse_weighted_combine(outputs, lses, return_lse=False, is_lse_base_on_e=True)
     merge_dcp_outputs(output_recv, lse_recv, token_dim)   (head- or token-scattered layouts)
+    lse_weighted_combine_varlen(outputs, lses, seq_lens, query_start_loc, interleave=1, ...)
     pack(cp_attn_out, cp_attn_lse, world_size)
     unpack_combine(recv_buf, return_lse=False, is_lse_base_on_e=True)
 """
@@ -30,8 +32,9 @@ import torch
 from . import _build
 
 __all__ = [
-    "DCPError", "library", "dcp_lse_pack_dim", "dcp_pack", "dcp_lse_combine", "dcp_unpack_combine",
-    "dcp_last_error", "dcp_version", "lse_weighted_combine", "merge_dcp_outputs", "pack", "unpack_combine",
+    "DCPError", "library", "dcp_lse_pack_dim", "dcp_pack", "dcp_lse_combine", "dcp_lse_combine_varlen",
+    "dcp_unpack_combine", "dcp_last_error", "dcp_version", "lse_weighted_combine", "lse_weighted_combine_varlen",
+    "merge_dcp_outputs", "pack", "unpack_combine",
     "DTYPE_CODES",
 ]
 
@@ -71,6 +74,9 @@ def library() -> ctypes.CDLL:
                                                         _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64,
                                                         _i32, _i32, _i32, _ptr]
                 lib.dcp_lse_combine_strided.restype = _i32
+                lib.dcp_lse_combine_varlen.argtypes = [_ptr, _ptr, _ptr, _ptr, _i32, _i64, _i64, _i64, _i64, _i64,
+                                                       _ptr, _ptr, _i32, _i32, _i32, _i32, _i32, _ptr]
+                lib.dcp_lse_combine_varlen.restype = _i32
                 lib.dcp_unpack_combine.argtypes = [_ptr, _ptr, _ptr, _i32, _i64, _i64, _i64, _i64, _i32, _i32, _i32,
                                                    _ptr]
                 lib.dcp_unpack_combine.restype = _i32
@@ -193,6 +199,39 @@ def dcp_lse_combine(outputs: torch.Tensor, lses: torch.Tensor, result: torch.Ten
             _code(outputs.dtype), int(bool(is_lse_base_on_e)), int(bool(return_lse)), _stream(dev, stream)))
 
 
+def dcp_lse_combine_varlen(outputs: torch.Tensor, lses: torch.Tensor, result: torch.Tensor, seq_lens: torch.Tensor,
+                           query_start_loc: torch.Tensor, global_lse: torch.Tensor | None = None,
+                           interleave: int = 1, is_lse_base_on_e: bool = True, return_lse: bool = False,
+                           stream=None) -> None:
+    """Variable-length combine: outputs [N, B, H, D] + lses [N, B, H] fp32 -> result [B, H, D], where
+    token b of request r (query_start_loc[r] <= b < query_start_loc[r+1]) combines only the shards
+    n with n * interleave < seq_lens[r]; rows of the other shards are never read.  seq_lens
+    [R] and query_start_loc [R + 1] are int32 tensors on the same device.  Shards may be
+    capacity-strided (outputs.stride(0) >= B*H*D); dims 1..3 must be contiguous."""
+    dev = _cuda(outputs, lses, result, global_lse, seq_lens, query_start_loc)
+    N, B, H, D = outputs.shape
+    if lses.shape != (N, B, H) or lses.dtype != torch.float32:
+        raise ValueError(f"lses must be fp32 [{N}, {B}, {H}], got {lses.dtype} {tuple(lses.shape)}")
+    if (outputs.stride()[1:] != (H * D, D, 1) and B * H > 1) or lses.stride()[1:] != (H, 1):
+        raise ValueError("outputs and lses must be contiguous within a shard")
+    if result.shape != (B, H, D) or result.dtype != outputs.dtype or not result.is_contiguous():
+        raise ValueError(f"result must be a contiguous [{B}, {H}, {D}] tensor of the output dtype")
+    if return_lse and (global_lse is None or global_lse.shape != (B, H) or global_lse.dtype != torch.float32
+                       or not global_lse.is_contiguous()):
+        raise ValueError("return_lse needs a contiguous fp32 [B, H] global_lse")
+    R = seq_lens.numel()
+    for t, n, what in ((seq_lens, R, "seq_lens"), (query_start_loc, R + 1, "query_start_loc")):
+        if t.dtype != torch.int32 or t.dim() != 1 or t.numel() != n or not t.is_contiguous():
+            raise ValueError(f"{what} must be a contiguous 1-D int32 tensor of {n} entries")
+    with torch.cuda.device(dev):
+        _check(library().dcp_lse_combine_varlen(
+            outputs.data_ptr(), lses.data_ptr(), result.data_ptr(),
+            global_lse.data_ptr() if (return_lse and global_lse is not None) else None,
+            N, B, H, D, outputs.stride(0) if N > 1 else B * H * D, lses.stride(0) if N > 1 else B * H,
+            seq_lens.data_ptr() if R else None, query_start_loc.data_ptr(), R, int(interleave),
+            _code(outputs.dtype), int(bool(is_lse_base_on_e)), int(bool(return_lse)), _stream(dev, stream)))
+
+
 def dcp_unpack_combine(recv_buf: torch.Tensor, result: torch.Tensor, global_lse: torch.Tensor | None = None,
                        is_lse_base_on_e: bool = True, return_lse: bool = False, stream=None) -> None:
     """recv_buf [N, B, Hr, D + P] -> result [B, Hr, D] (+ global_lse [B, Hr] fp32)."""
@@ -223,6 +262,20 @@ def lse_weighted_combine(outputs: torch.Tensor, lses: torch.Tensor, return_lse: 
     result = torch.empty((B, H, D), dtype=outputs.dtype, device=outputs.device)
     glse = torch.empty((B, H), dtype=torch.float32, device=outputs.device) if return_lse else None
     dcp_lse_combine(outputs, lses, result, glse, is_lse_base_on_e=is_lse_base_on_e, return_lse=return_lse)
+    return (result, glse) if return_lse else result
+
+
+def lse_weighted_combine_varlen(outputs: torch.Tensor, lses: torch.Tensor, seq_lens: torch.Tensor,
+                                query_start_loc: torch.Tensor, interleave: int = 1, return_lse: bool = False,
+                                is_lse_base_on_e: bool = True):
+    """The receive-side reduce with the batch's request metadata (seq_lens [R], query_start_loc
+    [R + 1], int32 on the device): shards that hold no KV of a token's request are skipped,
+    tokens outside every request give 0 (and LSE -inf).  Returns [B, H, D] (and [B, H] fp32)."""
+    N, B, H, D = outputs.shape
+    result = torch.empty((B, H, D), dtype=outputs.dtype, device=outputs.device)
+    glse = torch.empty((B, H), dtype=torch.float32, device=outputs.device) if return_lse else None
+    dcp_lse_combine_varlen(outputs, lses, result, seq_lens, query_start_loc, glse, interleave=interleave,
+                           is_lse_base_on_e=is_lse_base_on_e, return_lse=return_lse)
     return (result, glse) if return_lse else result
 
 

@@ -138,10 +138,10 @@ int cached_resident_ctas(K kernel, InstanceCache &ic, int threads, size_t smem) 
     return n;
 }
 
-template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS, bool UNIFORM>
+template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS, bool UNIFORM, bool VARLEN>
 int32_t launch_combine(const dcp::CombineArgs &a, cudaStream_t stream) {
     const char *fn = PACKED ? "dcp_unpack_combine" : "dcp_lse_combine";
-    auto kernel = dcp::combine_kernel<T, G, CPL, NB, PACKED, MIN_CTAS, UNIFORM>;
+    auto kernel = dcp::combine_kernel<T, G, CPL, NB, PACKED, MIN_CTAS, UNIFORM, VARLEN>;
     static InstanceCache ic;
     constexpr int kUnitsPerWarp = 32 / G;
     constexpr int kWarps = dcp::kCombineThreads / 32;
@@ -161,22 +161,22 @@ int32_t launch_combine(const dcp::CombineArgs &a, cudaStream_t stream) {
 // bytes in flight per SM are set by how many warps fit.  Capping registers so
 // that 3 CTAs fit (2 for the four-slot shapes, which spill otherwise) measured
 // best on B200 for every shape.
-template <class T, int G, bool PACKED, bool UNIFORM>
+template <class T, int G, bool PACKED, bool UNIFORM, bool VARLEN>
 int32_t launch_cpl(dcp::CombineArgs a, int cpl, cudaStream_t stream) {
     switch (cpl) {
-        case 1: return launch_combine<T, G, 1, 8, PACKED, 3, UNIFORM>(a, stream);
-        case 2: return launch_combine<T, G, 2, 4, PACKED, 3, UNIFORM>(a, stream);
-        default: return launch_combine<T, G, 4, 2, PACKED, 2, UNIFORM>(a, stream);
+        case 1: return launch_combine<T, G, 1, 8, PACKED, 3, UNIFORM, VARLEN>(a, stream);
+        case 2: return launch_combine<T, G, 2, 4, PACKED, 3, UNIFORM, VARLEN>(a, stream);
+        default: return launch_combine<T, G, 4, 2, PACKED, 2, UNIFORM, VARLEN>(a, stream);
     }
 }
 
-template <class T, bool PACKED, bool UNIFORM>
+template <class T, bool PACKED, bool UNIFORM, bool VARLEN = false>
 int32_t launch_g(dcp::CombineArgs a, int G, int cpl, cudaStream_t stream) {
     switch (G) {
-        case 4: return launch_cpl<T, 4, PACKED, UNIFORM>(a, cpl, stream);
-        case 8: return launch_cpl<T, 8, PACKED, UNIFORM>(a, cpl, stream);
-        case 16: return launch_cpl<T, 16, PACKED, UNIFORM>(a, cpl, stream);
-        default: return launch_cpl<T, 32, PACKED, UNIFORM>(a, cpl, stream);
+        case 4: return launch_cpl<T, 4, PACKED, UNIFORM, VARLEN>(a, cpl, stream);
+        case 8: return launch_cpl<T, 8, PACKED, UNIFORM, VARLEN>(a, cpl, stream);
+        case 16: return launch_cpl<T, 16, PACKED, UNIFORM, VARLEN>(a, cpl, stream);
+        default: return launch_cpl<T, 32, PACKED, UNIFORM, VARLEN>(a, cpl, stream);
     }
 }
 
@@ -203,6 +203,7 @@ int32_t dispatch_combine(dcp::CombineArgs a, cudaStream_t stream) {
         if (uniform) return launch_g<T, true, true>(a, G, cpl, stream);
         return launch_g<T, true, false>(a, G, cpl, stream);
     } else {
+        if (a.varlen) return launch_g<T, false, false, true>(a, G, cpl, stream);
         return launch_g<T, false, false>(a, G, cpl, stream);
     }
 }
@@ -247,12 +248,21 @@ int32_t dcp_lse_pack_dim(int32_t dtype) {
 
 namespace {
 
+// Request metadata of a variable-length combine (on == false: every shard is read).
+struct Varlen {
+    bool on = false;
+    const int32_t *seq_lens = nullptr;
+    const int32_t *qsl = nullptr;
+    int32_t num_reqs = 0;
+    int32_t interleave = 1;
+};
+
 // The split-layout combine with every stride explicit (elements of each array).
 int32_t lse_combine_impl(const char *fn, const void *outputs, const float *lses, void *result, float *global_lse,
                          int32_t N, int64_t B, int64_t H, int64_t D, int64_t os_n, int64_t os_b, int64_t os_h,
                          int64_t ls_n, int64_t ls_b, int64_t ls_h, int64_t rs_b, int64_t rs_h, int64_t gs_b,
                          int64_t gs_h, int32_t dtype, int32_t is_lse_base_on_e, int32_t return_lse,
-                         void *cuda_stream) {
+                         void *cuda_stream, const Varlen &vl = Varlen{}) {
     int32_t st = check_common(fn, dtype, N, B, H, D);
     if (st != DCP_OK) return st;
     const int es = elem_size(dtype);
@@ -295,15 +305,17 @@ int32_t lse_combine_impl(const char *fn, const void *outputs, const float *lses,
     a.N = N;
     a.base_e = is_lse_base_on_e ? 1 : 0;
     a.return_lse = return_lse ? 1 : 0;
+    a.varlen = vl.on ? 1 : 0;
+    a.num_reqs = vl.num_reqs;
+    a.interleave = vl.interleave;
+    a.seq_lens = vl.seq_lens;
+    a.qsl = vl.qsl;
     return dispatch_dtype<false>(dtype, a, static_cast<cudaStream_t>(cuda_stream));
 }
 
-}  // namespace
-
-int32_t dcp_lse_combine(const void *outputs, const float *lses, void *result, float *global_lse, int32_t N, int64_t B,
-                        int64_t H, int64_t D, int64_t out_stride_n, int64_t lse_stride_n, int32_t dtype,
-                        int32_t is_lse_base_on_e, int32_t return_lse, void *cuda_stream) {
-    const char *fn = "dcp_lse_combine";
+// Layout checks of dcp_lse_combine (canonical [N, B, H, D] shards, shard strides free).
+int32_t check_split_layout(const char *fn, int32_t N, int64_t B, int64_t H, int64_t D, int64_t out_stride_n,
+                           int64_t lse_stride_n, int32_t dtype) {
     int32_t st = check_common(fn, dtype, N, B, H, D);
     if (st != DCP_OK) return st;
     if (out_stride_n < B * H * D)
@@ -315,6 +327,17 @@ int32_t dcp_lse_combine(const void *outputs, const float *lses, void *result, fl
     if ((out_stride_n * elem_size(dtype)) % 16 != 0)
         return fail(DCP_ERR_MISALIGNED, "%s: out_stride_n %lld elements is not a multiple of 16 bytes", fn,
                     (long long)out_stride_n);
+    return DCP_OK;
+}
+
+}  // namespace
+
+int32_t dcp_lse_combine(const void *outputs, const float *lses, void *result, float *global_lse, int32_t N, int64_t B,
+                        int64_t H, int64_t D, int64_t out_stride_n, int64_t lse_stride_n, int32_t dtype,
+                        int32_t is_lse_base_on_e, int32_t return_lse, void *cuda_stream) {
+    const char *fn = "dcp_lse_combine";
+    int32_t st = check_split_layout(fn, N, B, H, D, out_stride_n, lse_stride_n, dtype);
+    if (st != DCP_OK) return st;
     return lse_combine_impl(fn, outputs, lses, result, global_lse, N, B, H, D, out_stride_n, H * D, D, lse_stride_n,
                             H, 1, H * D, D, H, 1, dtype, is_lse_base_on_e, return_lse, cuda_stream);
 }
@@ -329,6 +352,33 @@ int32_t dcp_lse_combine_strided(const void *outputs, const float *lses, void *re
                             out_stride_b, out_stride_h, lse_stride_n, lse_stride_b, lse_stride_h, result_stride_b,
                             result_stride_h, glse_stride_b, glse_stride_h, dtype, is_lse_base_on_e, return_lse,
                             cuda_stream);
+}
+
+int32_t dcp_lse_combine_varlen(const void *outputs, const float *lses, void *result, float *global_lse, int32_t N,
+                               int64_t B, int64_t H, int64_t D, int64_t out_stride_n, int64_t lse_stride_n,
+                               const int32_t *seq_lens, const int32_t *query_start_loc, int32_t num_reqs,
+                               int32_t interleave, int32_t dtype, int32_t is_lse_base_on_e, int32_t return_lse,
+                               void *cuda_stream) {
+    const char *fn = "dcp_lse_combine_varlen";
+    int32_t st = check_split_layout(fn, N, B, H, D, out_stride_n, lse_stride_n, dtype);
+    if (st != DCP_OK) return st;
+    if (num_reqs < 0) return fail(DCP_ERR_INVALID_ARG, "%s: negative request count %d", fn, (int)num_reqs);
+    if (interleave < 1) return fail(DCP_ERR_INVALID_ARG, "%s: interleave %d < 1", fn, (int)interleave);
+    if (num_reqs > 0 && B > 0) {
+        if (!seq_lens || !query_start_loc)
+            return fail(DCP_ERR_INVALID_ARG, "%s: seq_lens and query_start_loc are needed for %d requests", fn,
+                        (int)num_reqs);
+        if (!aligned(seq_lens, 4) || !aligned(query_start_loc, 4))
+            return fail(DCP_ERR_MISALIGNED, "%s: seq_lens and query_start_loc must be 4-byte aligned", fn);
+    }
+    Varlen vl;
+    vl.on = true;
+    vl.seq_lens = seq_lens;
+    vl.qsl = query_start_loc;
+    vl.num_reqs = num_reqs;
+    vl.interleave = interleave;
+    return lse_combine_impl(fn, outputs, lses, result, global_lse, N, B, H, D, out_stride_n, H * D, D, lse_stride_n,
+                            H, 1, H * D, D, H, 1, dtype, is_lse_base_on_e, return_lse, cuda_stream, vl);
 }
 
 int32_t dcp_unpack_combine(const void *recv_buf, void *result, float *global_lse, int32_t N, int64_t B, int64_t Hr,

@@ -188,7 +188,100 @@ struct CombineArgs {
     int32_t N;
     int32_t base_e;
     int32_t return_lse;
+    // split layout, variable length (varlen != 0, the VARLEN kernels): token b belongs to the request r
+    // with qsl[r] <= b < qsl[r + 1] (num_reqs + 1 non-decreasing entries); shard n
+    // holds KV of that request iff n * interleave < seq_lens[r].  A shard without
+    // KV counts as LSE -inf and its row is not read; a token outside every request
+    // combines no shard at all.
+    int32_t varlen;
+    int32_t num_reqs;
+    int32_t interleave;
+    const int32_t *seq_lens;
+    const int32_t *qsl;
 };
+
+// Variable-length combine: the shards that hold KV for a token are shards [0, k) of its
+// request, k = ceil(seq / interleave) capped at N (under interleaved sharding, blocks of
+// `interleave` positions dealt round-robin, shard n holds positions iff
+// n * interleave < seq); a token outside every request has none.
+__device__ __forceinline__ int varlen_held_shards(const CombineArgs &a, int32_t seq) {
+    if (seq <= 0) return 0;
+    const int32_t k = (seq - 1) / a.interleave + 1;
+    return k < a.N ? k : a.N;
+}
+
+// First of the G consecutive requests a row's first probe round reads for token b: the
+// token's interpolated request b * R / qsl[R] (r_per_token = R / qsl[R]) sits in the
+// middle of the window.  Lane jj probes clamp(window + jj, 0, R - 1).
+template <int G>
+__device__ __forceinline__ int64_t varlen_window(int64_t b, int R, int64_t qsl_end, float r_per_token) {
+    const int64_t guess = b < qsl_end ? (int64_t)((float)b * r_per_token) : (int64_t)R;
+    return guess - (G / 2 - 1);
+}
+
+__device__ __forceinline__ int clamp_req(int64_t q, int R) { return (int)(q < 0 ? 0 : q > R - 1 ? R - 1 : q); }
+
+// Shards holding KV for token b (0 for an inactive row): shards [0, k) of the request r
+// with qsl[r] <= b < qsl[r + 1], k = ceil(seq_lens[r] / interleave) capped at N; 0 when
+// b lies in no request.
+// The G lanes of a row search qsl together.  Each round every lane probes one position
+// (reading qsl and seq_lens there), a vote counts the probes <= b, and the range left for
+// the first start > b shrinks to the gap between two neighbouring probes.  Round 0 probes
+// the G consecutive requests of varlen_window (plain decode, where request r is token r,
+// ends there) and takes its reads from q0 / s0, fetched one task ahead; further rounds
+// split the range evenly, (G+1)-ary.  seq_lens[r] comes from the lane that probed r last
+// (else it is read).  All 32 lanes call this (it votes); every read stays inside
+// qsl[0..R - 1] and seq_lens[0..R), and it ends after at most 64 rounds whatever qsl
+// holds.  qsl_end = qsl[R]; full_seq = (N - 1) * interleave.
+template <int G>
+__device__ __forceinline__ int varlen_shards(const CombineArgs &a, int64_t b, bool active_row, int j, int64_t qsl_end,
+                                             float r_per_token, int64_t full_seq, int32_t q0, int32_t s0) {
+    const int R = a.num_reqs;
+    const int lane = threadIdx.x & 31;
+    const unsigned gmask = (G == 32 ? 0xffffffffu : ((1u << G) - 1u)) << (lane & (32 - G));
+    const bool searched = active_row && R > 0 && b < qsl_end;
+    // round 0
+    const int64_t window = varlen_window<G>(b, R, qsl_end, r_per_token);
+    int last_p = clamp_req(window + j, R);
+    int32_t last_s = s0;
+    const int c0 = __popc(__ballot_sync(0xffffffffu, searched && (int64_t)q0 <= b) & gmask);
+    // the first r in [0, R) with qsl[r] > b (R if none) lies in [lo, hi]
+    int lo = 0, hi = 0;
+    if (searched) {
+        lo = c0 == 0 ? 0 : clamp_req(window + c0 - 1, R) + 1;
+        hi = c0 == G ? R : clamp_req(window + c0, R);
+        lo = lo < hi ? lo : hi;  // lo > hi only when qsl is not non-decreasing
+    }
+    // further rounds, when the window missed
+    for (int round = 1; round < 64 && __any_sync(0xffffffffu, lo < hi); ++round) {
+        const bool active = lo < hi;  // the same for the G lanes of a row
+        auto probe = [&](int jj) -> int {
+            const int64_t q = lo + ((int64_t)(jj + 1) * (hi - lo)) / (G + 1);
+            return (int)(q > hi - 1 ? hi - 1 : q);
+        };
+        bool le = false;
+        if (active) {
+            last_p = probe(j);
+            le = (int64_t)__ldg(a.qsl + last_p) <= b;
+            last_s = __ldg(a.seq_lens + last_p);
+        }
+        const int c = __popc(__ballot_sync(0xffffffffu, le) & gmask);
+        if (active) {
+            const int nlo = c == 0 ? lo : probe(c - 1) + 1;
+            const int nhi = c == G ? hi : probe(c);
+            hi = nhi;
+            lo = nlo < nhi ? nlo : nhi;
+        }
+    }
+    // b < qsl_end was required, so lo >= 1 means b lies in request lo - 1
+    const int r = searched ? lo - 1 : -1;
+    const unsigned hit = __ballot_sync(0xffffffffu, r >= 0 && last_p == r) & gmask;
+    int32_t seq = __shfl_sync(0xffffffffu, last_s, hit ? __ffs(hit) - 1 : lane);
+    if (r < 0) return 0;
+    if (!hit) seq = __ldg(a.seq_lens + r);
+    if ((int64_t)seq > full_seq) return a.N;  // the usual case: KV on every shard
+    return varlen_held_shards(a, seq);
+}
 
 // The 4 words that start at word q (0..3) of the 8-word window (lo, hi).
 __device__ __forceinline__ Words<4> funnel_words(const Words<4> &lo, const Words<4> &hi, int q) {
@@ -241,7 +334,7 @@ __host__ __device__ constexpr size_t combine_smem_bytes(int units_per_warp, int 
 // output chunk c is elements 2q/e.. of sum c and the first ones of sum c+1 (from
 // the next lane, or, for the last chunk, the weighted sum of the tail chunks,
 // formed in phase 1 and reduced over the lane group).
-template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS = 1, bool UNIFORM = false>
+template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS = 1, bool UNIFORM = false, bool VARLEN = false>
 __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(const CombineArgs a) {
     constexpr int kUnitsPerWarp = 32 / G;
     constexpr int kWarps = kCombineThreads / 32;
@@ -258,11 +351,38 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
     float *sw = reinterpret_cast<float *>(s_dyn + (PACKED ? (size_t)kWarps * kUnitsPerWarp * a.N : 0)) +
                 (size_t)slot_base * a.N;
     const int64_t tasks = (a.units + kUnitsPerWarp - 1) / kUnitsPerWarp;
+    // VARLEN: the first search round's reads for each lane's next token are copied into
+    // shared memory one task ahead (two buffers, alternating), so they never wait.
+    __shared__ int32_t s_probe[VARLEN ? 2 : 1][VARLEN ? 2 * kCombineThreads : 1];
+    int64_t qsl_end = 0;
+    float r_per_token = 0.0f;
+    const int64_t full_seq = (int64_t)(a.N - 1) * a.interleave;
+    int buf = 0;
+    auto fetch_probe = [&](int64_t t, int into) {
+        const int64_t uu = t * kUnitsPerWarp + ul;
+        if (uu < a.units && a.num_reqs > 0) {
+            const int64_t bb = (int64_t)div_magic((uint64_t)uu, a.heads_magic);
+            const int p = clamp_req(varlen_window<G>(bb, a.num_reqs, qsl_end, r_per_token) + j, a.num_reqs);
+            cp_async_word(reinterpret_cast<uint32_t *>(&s_probe[into][2 * threadIdx.x]),
+                          reinterpret_cast<const uint32_t *>(a.qsl + p));
+            cp_async_word(reinterpret_cast<uint32_t *>(&s_probe[into][2 * threadIdx.x + 1]),
+                          reinterpret_cast<const uint32_t *>(a.seq_lens + p));
+        }
+        cp_async_commit();
+    };
+    if constexpr (VARLEN) {
+        if (a.num_reqs > 0) {
+            qsl_end = __ldg(a.qsl + a.num_reqs);
+            if (qsl_end > 0) r_per_token = (float)a.num_reqs / (float)qsl_end;
+        }
+        fetch_probe((int64_t)blockIdx.x * kWarps + warp, 0);
+    }
 
     for (int64_t task = (int64_t)blockIdx.x * kWarps + warp; task < tasks; task += (int64_t)gridDim.x * kWarps) {
         const int64_t u = task * kUnitsPerWarp + ul;
         const bool valid = u < a.units;
         int64_t row, lse_off, res_off, glse_off;
+        int nk = a.N;  // shards [0, nk) are read; the rest weigh 0
         if constexpr (PACKED) {
             row = u * a.row_pitch_w;
             res_off = u * a.data_w;
@@ -275,6 +395,12 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
             lse_off = b * a.lse_sb + h * a.lse_sh;
             res_off = b * a.res_sb_w + h * a.res_sh_w;
             glse_off = b * a.glse_sb + h * a.glse_sh;
+            if constexpr (VARLEN) {
+                cp_async_wait<0>();
+                const int32_t q0 = s_probe[buf][2 * threadIdx.x];
+                const int32_t s0 = s_probe[buf][2 * threadIdx.x + 1];
+                nk = varlen_shards<G>(a, b, valid, j, qsl_end, r_per_token, full_seq, q0, s0);
+            }
         }
 
         int c[CPL];
@@ -297,7 +423,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
                 qv[i] = (int)(w0 & 3);
 #pragma unroll
                 for (int k = 0; k < CPL; ++k) {
-                    if (n0 + i < a.N && act[k]) {
+                    if (n0 + i < nk && act[k]) {
                         x[i][k] = load_stream<4>(a.src + wa + 4 * c[k]);
                     } else {
 #pragma unroll
@@ -309,12 +435,16 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
 
         set_pass(0);
         issue(0);
+        if constexpr (VARLEN) {
+            buf ^= 1;
+            fetch_probe(task + (int64_t)gridDim.x * kWarps, buf);
+        }
 
         // ---- phase 1: weights of the N shards --------------------------------
         float lmax = -INFINITY;
         for (int n = j; n < a.N; n += G) {
             float l = -INFINITY;
-            if (valid) {
+            if (valid && n < nk) {
                 uint32_t bits;
                 if constexpr (PACKED) {
                     const int64_t w0 = (int64_t)n * a.shard_stride_w + row;

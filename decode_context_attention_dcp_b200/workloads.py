@@ -76,6 +76,14 @@ class CombineWorkload:
         wr = units * (self.D * self.elem_bytes + (4 if self.return_lse else 0))
         return rd + wr
 
+    def varlen_combine_bytes(self, shards_read: int, num_reqs: int) -> int:
+        """Algorithmic HBM bytes of one variable-length combine in which `shards_read` (token,
+        shard) pairs hold KV: those rows and LSEs (Hr heads each) are read, every result row is
+        written (+ the global LSE), and the request metadata (seq_lens, query_start_loc) read."""
+        rd = shards_read * self.Hr * (self.D * self.elem_bytes + 4) + 4 * (2 * num_reqs + 1)
+        wr = self.B * self.Hr * (self.D * self.elem_bytes + (4 if self.return_lse else 0))
+        return rd + wr
+
     def pack_bytes(self) -> int:
         """Algorithmic HBM bytes of one pack: each of the B*H rows (D elements + fp32 LSE) read once
         and written once."""
@@ -196,3 +204,39 @@ def attention_inputs(c: AttentionCase) -> tuple[torch.Tensor, torch.Tensor, torc
     k = torch.empty((c.B, c.L, c.H, c.D)).normal_(0.0, 1.0, generator=gen).to(dt)
     v = torch.empty((c.B, c.L, c.H, c.D)).normal_(0.0, 1.0, generator=gen).to(dt)
     return q, k, v
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeBatch:
+    """Request metadata of a decode batch of B token slots: requests of 1..max_q query tokens
+    each (1 = plain decode, more = speculative tokens) laid end to end from token 0, then
+    `pad` padding slots that belong to no request.  Each request's KV length is drawn from a
+    mix: with probability p_short uniform in [0, short_max] (0 = no KV at all), else uniform
+    in [short_max + 1, max_seq]."""
+
+    B: int
+    max_q: int = 1
+    pad: int = 0
+    p_short: float = 0.3
+    short_max: int = 16
+    max_seq: int = 8192
+    seed: int = 0
+
+
+def decode_batch(c: DecodeBatch) -> tuple[torch.Tensor, torch.Tensor]:
+    """(seq_lens [R] int32, query_start_loc [R + 1] int32) on the CPU, with
+    query_start_loc[R] = B - pad.  Draws: per request its query length (uniform 1..max_q,
+    cut at the last real slot), then per request one uniform u for the length class and one
+    integer for the length."""
+    gen = torch.Generator().manual_seed(c.seed)
+    real = max(0, c.B - c.pad)
+    starts = [0]
+    while starts[-1] < real:
+        q = int(torch.randint(1, c.max_q + 1, (1,), generator=gen))
+        starts.append(min(real, starts[-1] + q))
+    R = len(starts) - 1
+    u = torch.rand(R, generator=gen)
+    short = torch.randint(0, c.short_max + 1, (R,), generator=gen)
+    long = torch.randint(c.short_max + 1, c.max_seq + 1, (R,), generator=gen)
+    seq_lens = torch.where(u < c.p_short, short, long).to(torch.int32)
+    return seq_lens, torch.tensor(starts, dtype=torch.int32)

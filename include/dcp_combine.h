@@ -11,6 +11,7 @@
  *   dcp_pack                 partial output + fp32 LSE -> one packed send buffer
  *   dcp_lse_combine          combine of separate output / LSE receive buffers
  *   dcp_lse_combine_strided  the same with any token / head layout
+ *   dcp_lse_combine_varlen   the same per request: shards without KV are skipped
  *   dcp_unpack_combine       combine read straight out of the packed buffer
  *
  * Defining passages (web pages, by title and section):
@@ -162,6 +163,43 @@ int32_t dcp_lse_combine_strided(const void *outputs, const float *lses, void *re
                                 int64_t result_stride_b, int64_t result_stride_h,
                                 int64_t glse_stride_b, int64_t glse_stride_h, int32_t dtype,
                                 int32_t is_lse_base_on_e, int32_t return_lse, void *cuda_stream);
+
+/*
+ * Variable-length combine of split receive buffers: the receive-side reduce of
+ * [DIRECT] (DirectDCPA2AWorkspace.lse_reduce), which also takes the batch's
+ * seq_lens and query_start_loc.  The page does not define what the reduce does
+ * with them; this library reads them as follows.
+ *   - Token b belongs to request r when query_start_loc[r] <= b <
+ *     query_start_loc[r + 1].  A token outside every request (padding) has no
+ *     context: its result row is 0 and its global LSE -inf.
+ *   - Shard n holds KV of request r when n * interleave < seq_lens[r]
+ *     (blocks of `interleave` KV positions dealt round-robin to the N ranks, as
+ *     in [ASCEND] AscendSFACPMetadataBuilder._get_dcp_local_seq_lens).  A shard
+ *     that holds none counts as LSE -inf and its output row is NOT read: it may
+ *     hold anything, NaN included.
+ *   - Everything else is the [COMBINE] rule set, as dcp_lse_combine.
+ *
+ * outputs, lses, result, global_lse, out_stride_n, lse_stride_n: as
+ *             dcp_lse_combine.
+ * seq_lens    [num_reqs] int32 DEVICE array: KV length of each request, >= 0
+ *             (a value <= 0 means no shard holds KV).
+ * query_start_loc  [num_reqs + 1] int32 DEVICE array, non-decreasing: the first
+ *             token of each request, then the end of the last one.  Values that
+ *             are not non-decreasing give unspecified results but no access
+ *             outside the two arrays.
+ * num_reqs    >= 0; with 0 every token is padding and the arrays may be NULL.
+ * interleave  >= 1: KV positions per round-robin block (1 = token interleave).
+ *
+ * Requirements: as dcp_lse_combine; seq_lens and query_start_loc non-NULL
+ * (when num_reqs > 0 and B > 0) and 4-byte aligned, else DCP_ERR_INVALID_ARG /
+ * DCP_ERR_MISALIGNED.
+ */
+int32_t dcp_lse_combine_varlen(const void *outputs, const float *lses, void *result, float *global_lse,
+                               int32_t N, int64_t B, int64_t H, int64_t D,
+                               int64_t out_stride_n, int64_t lse_stride_n,
+                               const int32_t *seq_lens, const int32_t *query_start_loc,
+                               int32_t num_reqs, int32_t interleave, int32_t dtype,
+                               int32_t is_lse_base_on_e, int32_t return_lse, void *cuda_stream);
 
 /*
  * Fused unpack + combine over the packed receive buffer ([A2A], the step

@@ -175,3 +175,31 @@ def test_strided_rejections(lib):
     assert _strided(lib, glse=None) == INVALID
     assert _strided(lib, B=1 << 22, H=1 << 10) == INVALID  # 2^32 result rows
     assert "dcp_lse_combine_strided" in dcp.dcp_last_error()
+
+
+def _varlen(lib, **kw):
+    a = dict(outputs=A, lses=A, result=A, glse=A, N=2, B=4, H=8, D=128, sn=None, ln=None, seq=A, qsl=A, R=3,
+             inter=1, dtype=0, ret=1)
+    a.update(kw)
+    sn = a["sn"] if a["sn"] is not None else a["B"] * a["H"] * a["D"]
+    ln = a["ln"] if a["ln"] is not None else a["B"] * a["H"]
+    return lib.dcp_lse_combine_varlen(a["outputs"], a["lses"], a["result"], a["glse"], a["N"], a["B"], a["H"],
+                                      a["D"], sn, ln, a["seq"], a["qsl"], a["R"], a["inter"], a["dtype"], 1,
+                                      a["ret"], None)
+
+
+def test_varlen_rejections(lib):
+    assert _varlen(lib, B=0) == OK
+    assert _varlen(lib, dtype=3) == DTYPE
+    assert _varlen(lib, N=65) == INVALID
+    assert _varlen(lib, sn=4 * 8 * 128 - 8) == INVALID
+    assert _varlen(lib, sn=4 * 8 * 128 + 4) == MISALIGNED
+    assert _varlen(lib, R=-1) == INVALID
+    assert _varlen(lib, inter=0) == INVALID
+    assert _varlen(lib, seq=None) == INVALID
+    assert _varlen(lib, qsl=None) == INVALID
+    assert _varlen(lib, seq=A + 2) == MISALIGNED
+    assert _varlen(lib, qsl=A + 1) == MISALIGNED
+    assert _varlen(lib, outputs=A + 8) == MISALIGNED
+    assert _varlen(lib, glse=None, ret=1) == INVALID
+    assert "dcp_lse_combine_varlen" in dcp.dcp_last_error()
