@@ -210,52 +210,39 @@ __device__ __forceinline__ int varlen_held_shards(const CombineArgs &a, int32_t 
     return k < a.N ? k : a.N;
 }
 
-// First of the G consecutive requests a row's first probe round reads for token b: the
-// token's interpolated request b * R / qsl[R] (r_per_token = R / qsl[R]) sits in the
-// middle of the window.  Lane jj probes clamp(window + jj, 0, R - 1).
-template <int G>
-__device__ __forceinline__ int64_t varlen_window(int64_t b, int R, int64_t qsl_end, float r_per_token) {
-    const int64_t guess = b < qsl_end ? (int64_t)((float)b * r_per_token) : (int64_t)R;
-    return guess - (G / 2 - 1);
-}
-
 __device__ __forceinline__ int clamp_req(int64_t q, int R) { return (int)(q < 0 ? 0 : q > R - 1 ? R - 1 : q); }
 
-// Shards holding KV for token b (0 for an inactive row): shards [0, k) of the request r
-// with qsl[r] <= b < qsl[r + 1], k = ceil(seq_lens[r] / interleave) capped at N; 0 when
-// b lies in no request.
-// The G lanes of a row search qsl together.  Each round every lane probes one position
-// (reading qsl and seq_lens there), a vote counts the probes <= b, and the range left for
-// the first start > b shrinks to the gap between two neighbouring probes.  Round 0 probes
-// the G consecutive requests of varlen_window (plain decode, where request r is token r,
-// ends there) and takes its reads from q0 / s0, fetched one task ahead; further rounds
-// split the range evenly, (G+1)-ary.  seq_lens[r] comes from the lane that probed r last
+// The request a token's position interpolates to: b * R / qsl[R] (r_per_token = R / qsl[R]),
+// clamped to [0, R - 1].  Exact for plain decode (request r is token r) and for any batch
+// whose requests all have the same number of query tokens.
+__device__ __forceinline__ int varlen_guess(int64_t b, int R, int64_t qsl_end, float r_per_token) {
+    return clamp_req(b < qsl_end ? (int64_t)((float)b * r_per_token) : (int64_t)R - 1, R);
+}
+
+// The request r with qsl[r] <= b < qsl[r + 1] for the rows whose `active` is set (-1 if
+// none), and its seq_lens entry.  The G lanes of a row search together.  Each round every
+// lane probes one position (reading qsl and seq_lens there), a vote counts the probes <= b,
+// and the range left for the first start > b shrinks to the gap between two neighbouring
+// probes.  Round 0 probes the G consecutive requests around varlen_guess; later rounds split
+// the range evenly, (G+1)-ary.  The seq_lens entry comes from the lane that probed r last
 // (else it is read).  All 32 lanes call this (it votes); every read stays inside
-// qsl[0..R - 1] and seq_lens[0..R), and it ends after at most 64 rounds whatever qsl
-// holds.  qsl_end = qsl[R]; full_seq = (N - 1) * interleave.
+// qsl[0..R - 1] and seq_lens[0..R), and it ends after at most 64 rounds whatever qsl holds.
+// An active row needs b < qsl_end = qsl[R].
 template <int G>
-__device__ __forceinline__ int varlen_shards(const CombineArgs &a, int64_t b, bool active_row, int j, int64_t qsl_end,
-                                             float r_per_token, int64_t full_seq, int32_t q0, int32_t s0) {
+__device__ __forceinline__ int varlen_search(const CombineArgs &a, int64_t b, bool active_row, int j,
+                                            int64_t qsl_end, float r_per_token, int32_t &seq) {
     const int R = a.num_reqs;
     const int lane = threadIdx.x & 31;
     const unsigned gmask = (G == 32 ? 0xffffffffu : ((1u << G) - 1u)) << (lane & (32 - G));
-    const bool searched = active_row && R > 0 && b < qsl_end;
-    // round 0
-    const int64_t window = varlen_window<G>(b, R, qsl_end, r_per_token);
-    int last_p = clamp_req(window + j, R);
-    int32_t last_s = s0;
-    const int c0 = __popc(__ballot_sync(0xffffffffu, searched && (int64_t)q0 <= b) & gmask);
+    const int64_t window = (int64_t)varlen_guess(b, R, qsl_end, r_per_token) - (G / 2 - 1);
     // the first r in [0, R) with qsl[r] > b (R if none) lies in [lo, hi]
-    int lo = 0, hi = 0;
-    if (searched) {
-        lo = c0 == 0 ? 0 : clamp_req(window + c0 - 1, R) + 1;
-        hi = c0 == G ? R : clamp_req(window + c0, R);
-        lo = lo < hi ? lo : hi;  // lo > hi only when qsl is not non-decreasing
-    }
-    // further rounds, when the window missed
-    for (int round = 1; round < 64 && __any_sync(0xffffffffu, lo < hi); ++round) {
+    int lo = 0, hi = active_row ? R : 0;
+    int last_p = -1;
+    int32_t last_s = 0;
+    for (int round = 0; round < 64 && __any_sync(0xffffffffu, lo < hi); ++round) {
         const bool active = lo < hi;  // the same for the G lanes of a row
         auto probe = [&](int jj) -> int {
+            if (round == 0) return clamp_req(window + jj, R);  // lo = 0, hi = R
             const int64_t q = lo + ((int64_t)(jj + 1) * (hi - lo)) / (G + 1);
             return (int)(q > hi - 1 ? hi - 1 : q);
         };
@@ -270,15 +257,39 @@ __device__ __forceinline__ int varlen_shards(const CombineArgs &a, int64_t b, bo
             const int nlo = c == 0 ? lo : probe(c - 1) + 1;
             const int nhi = c == G ? hi : probe(c);
             hi = nhi;
-            lo = nlo < nhi ? nlo : nhi;
+            lo = nlo < nhi ? nlo : nhi;  // nlo > nhi only when qsl is not non-decreasing
         }
     }
-    // b < qsl_end was required, so lo >= 1 means b lies in request lo - 1
-    const int r = searched ? lo - 1 : -1;
+    // b < qsl_end, so lo >= 1 means b lies in request lo - 1
+    const int r = active_row ? lo - 1 : -1;
     const unsigned hit = __ballot_sync(0xffffffffu, r >= 0 && last_p == r) & gmask;
-    int32_t seq = __shfl_sync(0xffffffffu, last_s, hit ? __ffs(hit) - 1 : lane);
-    if (r < 0) return 0;
-    if (!hit) seq = __ldg(a.seq_lens + r);
+    seq = __shfl_sync(0xffffffffu, last_s, hit ? __ffs(hit) - 1 : lane);
+    if (r >= 0 && !hit) seq = __ldg(a.seq_lens + r);
+    return r;
+}
+
+// Shards holding KV for token b (0 for an inactive row): shards [0, k) of its request,
+// k = ceil(seq / interleave) capped at N; 0 when b lies in no request.  q_lo, q_hi, s_g are
+// qsl[g], qsl[g + 1] and seq_lens[g] for g = varlen_guess(b), fetched one task ahead: when
+// request g holds b nothing else is read; otherwise the row's lanes run varlen_search.  All
+// 32 lanes call this.  full_seq = (N - 1) * interleave.
+template <int G>
+__device__ __forceinline__ int varlen_shards(const CombineArgs &a, int64_t b, bool active_row, int j, int64_t qsl_end,
+                                             float r_per_token, int64_t full_seq, int32_t q_lo, int32_t q_hi,
+                                             int32_t s_g) {
+    const bool searched = active_row && a.num_reqs > 0 && b < qsl_end;
+    bool found = searched && (int64_t)q_lo <= b && b < (int64_t)q_hi;
+    int32_t seq = s_g;
+    const bool need = searched && !found;
+    if (__any_sync(0xffffffffu, need)) {
+        int32_t s_r;
+        const int r = varlen_search<G>(a, b, need, j, qsl_end, r_per_token, s_r);
+        if (need) {
+            found = r >= 0;
+            seq = s_r;
+        }
+    }
+    if (!found) return 0;
     if ((int64_t)seq > full_seq) return a.N;  // the usual case: KV on every shard
     return varlen_held_shards(a, seq);
 }
@@ -351,22 +362,23 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
     float *sw = reinterpret_cast<float *>(s_dyn + (PACKED ? (size_t)kWarps * kUnitsPerWarp * a.N : 0)) +
                 (size_t)slot_base * a.N;
     const int64_t tasks = (a.units + kUnitsPerWarp - 1) / kUnitsPerWarp;
-    // VARLEN: the first search round's reads for each lane's next token are copied into
-    // shared memory one task ahead (two buffers, alternating), so they never wait.
-    __shared__ int32_t s_probe[VARLEN ? 2 : 1][VARLEN ? 2 * kCombineThreads : 1];
+    // VARLEN: for each row's next token, lane 0 of the row copies qsl[g], qsl[g + 1] and
+    // seq_lens[g] (g = varlen_guess) into shared memory one task ahead (two buffers,
+    // alternating), so the usual case waits on no global read.
+    __shared__ int32_t s_probe[VARLEN ? 2 : 1][VARLEN ? 3 * kWarps * kUnitsPerWarp : 1];
     int64_t qsl_end = 0;
     float r_per_token = 0.0f;
     const int64_t full_seq = (int64_t)(a.N - 1) * a.interleave;
     int buf = 0;
-    auto fetch_probe = [&](int64_t t, int into) {
+    auto fetch_guess = [&](int64_t t, int into) {
         const int64_t uu = t * kUnitsPerWarp + ul;
-        if (uu < a.units && a.num_reqs > 0) {
+        if (j == 0 && uu < a.units && a.num_reqs > 0) {
             const int64_t bb = (int64_t)div_magic((uint64_t)uu, a.heads_magic);
-            const int p = clamp_req(varlen_window<G>(bb, a.num_reqs, qsl_end, r_per_token) + j, a.num_reqs);
-            cp_async_word(reinterpret_cast<uint32_t *>(&s_probe[into][2 * threadIdx.x]),
-                          reinterpret_cast<const uint32_t *>(a.qsl + p));
-            cp_async_word(reinterpret_cast<uint32_t *>(&s_probe[into][2 * threadIdx.x + 1]),
-                          reinterpret_cast<const uint32_t *>(a.seq_lens + p));
+            const int g = varlen_guess(bb, a.num_reqs, qsl_end, r_per_token);
+            uint32_t *d = reinterpret_cast<uint32_t *>(&s_probe[into][3 * slot_base]);
+            cp_async_word(d, reinterpret_cast<const uint32_t *>(a.qsl + g));
+            cp_async_word(d + 1, reinterpret_cast<const uint32_t *>(a.qsl + g + 1));
+            cp_async_word(d + 2, reinterpret_cast<const uint32_t *>(a.seq_lens + g));
         }
         cp_async_commit();
     };
@@ -375,7 +387,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
             qsl_end = __ldg(a.qsl + a.num_reqs);
             if (qsl_end > 0) r_per_token = (float)a.num_reqs / (float)qsl_end;
         }
-        fetch_probe((int64_t)blockIdx.x * kWarps + warp, 0);
+        fetch_guess((int64_t)blockIdx.x * kWarps + warp, 0);
     }
 
     for (int64_t task = (int64_t)blockIdx.x * kWarps + warp; task < tasks; task += (int64_t)gridDim.x * kWarps) {
@@ -396,10 +408,10 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
             res_off = b * a.res_sb_w + h * a.res_sh_w;
             glse_off = b * a.glse_sb + h * a.glse_sh;
             if constexpr (VARLEN) {
-                cp_async_wait<0>();
-                const int32_t q0 = s_probe[buf][2 * threadIdx.x];
-                const int32_t s0 = s_probe[buf][2 * threadIdx.x + 1];
-                nk = varlen_shards<G>(a, b, valid, j, qsl_end, r_per_token, full_seq, q0, s0);
+                cp_async_wait<0>();  // lane 0's copies for this task
+                __syncwarp();
+                const int32_t *pr = &s_probe[buf][3 * slot_base];
+                nk = varlen_shards<G>(a, b, valid, j, qsl_end, r_per_token, full_seq, pr[0], pr[1], pr[2]);
             }
         }
 
@@ -437,7 +449,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
         issue(0);
         if constexpr (VARLEN) {
             buf ^= 1;
-            fetch_probe(task + (int64_t)gridDim.x * kWarps, buf);
+            fetch_guess(task + (int64_t)gridDim.x * kWarps, buf);
         }
 
         // ---- phase 1: weights of the N shards --------------------------------
