@@ -306,6 +306,24 @@ def run_sweep(args) -> int:
                             lambda: dcp.dcp_lse_combine_varlen(d_out, d_lse, res, d_seq, d_qsl, gl,
                                                                is_lse_base_on_e=w.is_lse_base_on_e,
                                                                return_lse=w.return_lse)))
+        if w.B >= 4096 or w is wl.MLA:
+            # a producer with S = 4 KV splits per rank: its split merge fused with the pack
+            # (dcp_combine_pack) against the merge into [B, H, D] followed by dcp_pack
+            S = 4
+            gen = torch.Generator(device="cuda").manual_seed(w.seed)
+            parts = torch.randn((S, w.B, w.H, w.D), generator=gen, device="cuda").to(d_out.dtype)
+            part_lse = torch.rand((S, w.B, w.H), generator=gen, device="cuda") * 20.0
+            merged = torch.empty((w.B, w.H, w.D), dtype=d_out.dtype, device="cuda")
+            merged_lse = torch.empty((w.B, w.H), dtype=torch.float32, device="cuda")
+            row = w.D * w.elem_bytes + 4
+            fused_bytes = w.B * w.H * (S * row + row)
+            kernels.append((f"dcp_combine_pack[S={S}]", fused_bytes,
+                            lambda: dcp.dcp_combine_pack(parts, part_lse, send, w.N)))
+
+            def two_step():
+                dcp.dcp_lse_combine(parts, part_lse, merged, merged_lse, return_lse=True)
+                dcp.dcp_pack(merged, merged_lse, send, w.N)
+            kernels.append((f"dcp_lse_combine+dcp_pack[S={S}]", fused_bytes + 2 * w.B * w.H * row, two_step))
         for name, nbytes, fn in kernels:
             for _ in range(3):
                 fn()
@@ -325,6 +343,7 @@ def run_sweep(args) -> int:
             print(f"| {w.name} | {w.N} | {w.B} | {w.Hr} | {w.D} | {w.dtype} | {name} | {nbytes} | {t * 1e3:.1f} | "
                   f"{gbs:.0f} | {gbs / peak:.3f} |", flush=True)
         del d_out, d_lse, recv, cp_out, cp_lse, res, gl, send, kernels
+        parts = part_lse = merged = merged_lse = None
         torch.cuda.empty_cache()
     return 0
 

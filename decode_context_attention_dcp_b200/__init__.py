@@ -12,6 +12,7 @@ Low-level calls (same names as the C ABI, caller-allocated outputs):
     dcp_pack(cp_attn_out, cp_attn_lse, send_buf, world_size)
     dcp_lse_combine(outputs, lses, result, global_lse=None, ...)
     dcp_lse_combine_varlen(outputs, lses, result, seq_lens, query_start_loc, ...)
+    dcp_combine_pack(partial_outputs, partial_lses, send_buf, world_size, ...)
     dcp_unpack_combine(recv_buf, result, global_lse=None, ...)
     dcp_lse_pack_dim(dtype), dcp_last_error()
 
@@ -20,6 +21,7 @@ Allocating helpers with the pages' argument conventions:
     merge_dcp_outputs(output_recv, lse_recv, token_dim)   (head- or token-scattered layouts)
     lse_weighted_combine_varlen(outputs, lses, seq_lens, query_start_loc, interleave=1, ...)
     pack(cp_attn_out, cp_attn_lse, world_size)
+    combine_pack(partial_outputs, partial_lses, world_size)   (split merge + pack in one pass)
     unpack_combine(recv_buf, return_lse=False, is_lse_base_on_e=True)
 """
 from __future__ import annotations
@@ -33,7 +35,7 @@ from . import _build
 
 __all__ = [
     "DCPError", "library", "dcp_lse_pack_dim", "dcp_pack", "dcp_lse_combine", "dcp_lse_combine_varlen",
-    "dcp_unpack_combine", "dcp_last_error", "dcp_version", "lse_weighted_combine", "lse_weighted_combine_varlen",
+    "dcp_combine_pack", "dcp_unpack_combine", "combine_pack", "dcp_last_error", "dcp_version", "lse_weighted_combine", "lse_weighted_combine_varlen",
     "merge_dcp_outputs", "pack", "unpack_combine",
     "DTYPE_CODES",
 ]
@@ -77,6 +79,9 @@ def library() -> ctypes.CDLL:
                 lib.dcp_lse_combine_varlen.argtypes = [_ptr, _ptr, _ptr, _ptr, _i32, _i64, _i64, _i64, _i64, _i64,
                                                        _ptr, _ptr, _i32, _i32, _i32, _i32, _i32, _ptr]
                 lib.dcp_lse_combine_varlen.restype = _i32
+                lib.dcp_combine_pack.argtypes = [_ptr, _ptr, _ptr, _i32, _i64, _i64, _i64, _i64, _i64, _i32, _i32,
+                                                 _i32, _ptr]
+                lib.dcp_combine_pack.restype = _i32
                 lib.dcp_unpack_combine.argtypes = [_ptr, _ptr, _ptr, _i32, _i64, _i64, _i64, _i64, _i32, _i32, _i32,
                                                    _ptr]
                 lib.dcp_unpack_combine.restype = _i32
@@ -232,6 +237,32 @@ def dcp_lse_combine_varlen(outputs: torch.Tensor, lses: torch.Tensor, result: to
             _code(outputs.dtype), int(bool(is_lse_base_on_e)), int(bool(return_lse)), _stream(dev, stream)))
 
 
+def dcp_combine_pack(partial_outputs: torch.Tensor, partial_lses: torch.Tensor, send_buf: torch.Tensor,
+                     world_size: int, is_lse_base_on_e: bool = True, stream=None) -> None:
+    """partial_outputs [S, B, H, D] + partial_lses [S, B, H] fp32 (a producer's S KV splits)
+    -> send_buf [world_size, B, H/world_size, D + P]: the merged rows, head-scattered, each
+    followed by its merged fp32 LSE.  Splits may be capacity-strided; dims 1..3 contiguous."""
+    dev = _cuda(partial_outputs, partial_lses, send_buf)
+    S, B, H, D = partial_outputs.shape
+    code = _code(partial_outputs.dtype)
+    if partial_lses.shape != (S, B, H) or partial_lses.dtype != torch.float32:
+        raise ValueError(f"partial_lses must be fp32 [{S}, {B}, {H}], got {partial_lses.dtype} "
+                         f"{tuple(partial_lses.shape)}")
+    if (partial_outputs.stride()[1:] != (H * D, D, 1) and B * H > 1) or partial_lses.stride()[1:] != (H, 1):
+        raise ValueError("partial_outputs and partial_lses must be contiguous within a split")
+    if world_size < 1 or H % world_size:
+        raise ValueError(f"H={H} heads do not split over world_size={world_size}")
+    P = library().dcp_lse_pack_dim(code)
+    want = (world_size, B, H // world_size, D + P)
+    if tuple(send_buf.shape) != want or send_buf.dtype != partial_outputs.dtype or not send_buf.is_contiguous():
+        raise ValueError(f"send_buf must be a contiguous {want} tensor of the output dtype")
+    with torch.cuda.device(dev):
+        _check(library().dcp_combine_pack(
+            partial_outputs.data_ptr(), partial_lses.data_ptr(), send_buf.data_ptr(), S, B, H, D,
+            partial_outputs.stride(0) if S > 1 else B * H * D, partial_lses.stride(0) if S > 1 else B * H,
+            int(world_size), code, int(bool(is_lse_base_on_e)), _stream(dev, stream)))
+
+
 def dcp_unpack_combine(recv_buf: torch.Tensor, result: torch.Tensor, global_lse: torch.Tensor | None = None,
                        is_lse_base_on_e: bool = True, return_lse: bool = False, stream=None) -> None:
     """recv_buf [N, B, Hr, D + P] -> result [B, Hr, D] (+ global_lse [B, Hr] fp32)."""
@@ -305,6 +336,19 @@ def pack(cp_attn_out: torch.Tensor, cp_attn_lse: torch.Tensor, world_size: int) 
     P = dcp_lse_pack_dim(cp_attn_out.dtype)
     send = torch.empty((world_size, B, H // world_size, D + P), dtype=cp_attn_out.dtype, device=cp_attn_out.device)
     dcp_pack(cp_attn_out, cp_attn_lse, send, world_size)
+    return send
+
+
+def combine_pack(partial_outputs: torch.Tensor, partial_lses: torch.Tensor, world_size: int,
+                 is_lse_base_on_e: bool = True) -> torch.Tensor:
+    """A producer's S split partials [S, B, H, D] (+ [S, B, H] fp32 LSEs) merged and packed in
+    one pass: the send buffer [world_size, B, H/world_size, D + P] that pack() would build from
+    the merged result and its LSE."""
+    S, B, H, D = partial_outputs.shape
+    P = dcp_lse_pack_dim(partial_outputs.dtype)
+    send = torch.empty((world_size, B, H // world_size, D + P), dtype=partial_outputs.dtype,
+                       device=partial_outputs.device)
+    dcp_combine_pack(partial_outputs, partial_lses, send, world_size, is_lse_base_on_e=is_lse_base_on_e)
     return send
 
 

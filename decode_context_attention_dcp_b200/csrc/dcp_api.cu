@@ -138,10 +138,10 @@ int cached_resident_ctas(K kernel, InstanceCache &ic, int threads, size_t smem) 
     return n;
 }
 
-template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS, bool UNIFORM, bool VARLEN>
+template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS, bool UNIFORM, bool VARLEN, bool PACK_OUT>
 int32_t launch_combine(const dcp::CombineArgs &a, cudaStream_t stream) {
-    const char *fn = PACKED ? "dcp_unpack_combine" : "dcp_lse_combine";
-    auto kernel = dcp::combine_kernel<T, G, CPL, NB, PACKED, MIN_CTAS, UNIFORM, VARLEN>;
+    const char *fn = PACKED ? "dcp_unpack_combine" : PACK_OUT ? "dcp_combine_pack" : "dcp_lse_combine";
+    auto kernel = dcp::combine_kernel<T, G, CPL, NB, PACKED, MIN_CTAS, UNIFORM, VARLEN, PACK_OUT>;
     static InstanceCache ic;
     constexpr int kUnitsPerWarp = 32 / G;
     constexpr int kWarps = dcp::kCombineThreads / 32;
@@ -161,22 +161,22 @@ int32_t launch_combine(const dcp::CombineArgs &a, cudaStream_t stream) {
 // bytes in flight per SM are set by how many warps fit.  Capping registers so
 // that 3 CTAs fit (2 for the four-slot shapes, which spill otherwise) measured
 // best on B200 for every shape.
-template <class T, int G, bool PACKED, bool UNIFORM, bool VARLEN>
+template <class T, int G, bool PACKED, bool UNIFORM, bool VARLEN, bool PACK_OUT>
 int32_t launch_cpl(dcp::CombineArgs a, int cpl, cudaStream_t stream) {
     switch (cpl) {
-        case 1: return launch_combine<T, G, 1, 8, PACKED, 3, UNIFORM, VARLEN>(a, stream);
-        case 2: return launch_combine<T, G, 2, 4, PACKED, 3, UNIFORM, VARLEN>(a, stream);
-        default: return launch_combine<T, G, 4, 2, PACKED, 2, UNIFORM, VARLEN>(a, stream);
+        case 1: return launch_combine<T, G, 1, 8, PACKED, 3, UNIFORM, VARLEN, PACK_OUT>(a, stream);
+        case 2: return launch_combine<T, G, 2, 4, PACKED, 3, UNIFORM, VARLEN, PACK_OUT>(a, stream);
+        default: return launch_combine<T, G, 4, 2, PACKED, 2, UNIFORM, VARLEN, PACK_OUT>(a, stream);
     }
 }
 
-template <class T, bool PACKED, bool UNIFORM, bool VARLEN = false>
+template <class T, bool PACKED, bool UNIFORM, bool VARLEN = false, bool PACK_OUT = false>
 int32_t launch_g(dcp::CombineArgs a, int G, int cpl, cudaStream_t stream) {
     switch (G) {
-        case 4: return launch_cpl<T, 4, PACKED, UNIFORM, VARLEN>(a, cpl, stream);
-        case 8: return launch_cpl<T, 8, PACKED, UNIFORM, VARLEN>(a, cpl, stream);
-        case 16: return launch_cpl<T, 16, PACKED, UNIFORM, VARLEN>(a, cpl, stream);
-        default: return launch_cpl<T, 32, PACKED, UNIFORM, VARLEN>(a, cpl, stream);
+        case 4: return launch_cpl<T, 4, PACKED, UNIFORM, VARLEN, PACK_OUT>(a, cpl, stream);
+        case 8: return launch_cpl<T, 8, PACKED, UNIFORM, VARLEN, PACK_OUT>(a, cpl, stream);
+        case 16: return launch_cpl<T, 16, PACKED, UNIFORM, VARLEN, PACK_OUT>(a, cpl, stream);
+        default: return launch_cpl<T, 32, PACKED, UNIFORM, VARLEN, PACK_OUT>(a, cpl, stream);
     }
 }
 
@@ -204,6 +204,7 @@ int32_t dispatch_combine(dcp::CombineArgs a, cudaStream_t stream) {
         return launch_g<T, true, false>(a, G, cpl, stream);
     } else {
         if (a.varlen) return launch_g<T, false, false, true>(a, G, cpl, stream);
+        if (a.pack_b > 0) return launch_g<T, false, false, false, true>(a, G, cpl, stream);
         return launch_g<T, false, false>(a, G, cpl, stream);
     }
 }
@@ -257,12 +258,19 @@ struct Varlen {
     int32_t interleave = 1;
 };
 
+// Packed output of a combine (dcp_combine_pack): B and heads per rank; on == false: plain rows.
+struct PackOut {
+    bool on = false;
+    int64_t B = 0;
+    int64_t Hr = 1;
+};
+
 // The split-layout combine with every stride explicit (elements of each array).
 int32_t lse_combine_impl(const char *fn, const void *outputs, const float *lses, void *result, float *global_lse,
                          int32_t N, int64_t B, int64_t H, int64_t D, int64_t os_n, int64_t os_b, int64_t os_h,
                          int64_t ls_n, int64_t ls_b, int64_t ls_h, int64_t rs_b, int64_t rs_h, int64_t gs_b,
                          int64_t gs_h, int32_t dtype, int32_t is_lse_base_on_e, int32_t return_lse,
-                         void *cuda_stream, const Varlen &vl = Varlen{}) {
+                         void *cuda_stream, const Varlen &vl = Varlen{}, const PackOut &po = PackOut{}) {
     int32_t st = check_common(fn, dtype, N, B, H, D);
     if (st != DCP_OK) return st;
     const int es = elem_size(dtype);
@@ -305,6 +313,9 @@ int32_t lse_combine_impl(const char *fn, const void *outputs, const float *lses,
     a.N = N;
     a.base_e = is_lse_base_on_e ? 1 : 0;
     a.return_lse = return_lse ? 1 : 0;
+    a.pack_b = po.on ? B : 0;
+    a.pack_hr = po.Hr;
+    a.pack_hr_magic = magic64((uint64_t)po.Hr);
     a.varlen = vl.on ? 1 : 0;
     a.num_reqs = vl.num_reqs;
     a.interleave = vl.interleave;
@@ -379,6 +390,29 @@ int32_t dcp_lse_combine_varlen(const void *outputs, const float *lses, void *res
     vl.interleave = interleave;
     return lse_combine_impl(fn, outputs, lses, result, global_lse, N, B, H, D, out_stride_n, H * D, D, lse_stride_n,
                             H, 1, H * D, D, H, 1, dtype, is_lse_base_on_e, return_lse, cuda_stream, vl);
+}
+
+int32_t dcp_combine_pack(const void *partial_outputs, const float *partial_lses, void *send_buf, int32_t S, int64_t B,
+                         int64_t H, int64_t D, int64_t out_stride_s, int64_t lse_stride_s, int32_t world_size,
+                         int32_t dtype, int32_t is_lse_base_on_e, void *cuda_stream) {
+    const char *fn = "dcp_combine_pack";
+    int32_t st = check_split_layout(fn, S, B, H, D, out_stride_s, lse_stride_s, dtype);
+    if (st != DCP_OK) return st;
+    if (world_size < 1 || world_size > DCP_MAX_SHARDS)
+        return fail(DCP_ERR_INVALID_ARG, "%s: world_size %d outside [1, %d]", fn, (int)world_size, DCP_MAX_SHARDS);
+    if (H % world_size != 0)
+        return fail(DCP_ERR_SHAPE, "%s: H=%lld heads do not split evenly over %d ranks", fn, (long long)H,
+                    (int)world_size);
+    if (B == 0) return ok();
+    if (!send_buf) return fail(DCP_ERR_INVALID_ARG, "%s: null buffer pointer", fn);
+    if (!aligned(send_buf, 16)) return fail(DCP_ERR_MISALIGNED, "%s: send_buf must be 16-byte aligned", fn);
+    PackOut po;
+    po.on = true;
+    po.B = B;
+    po.Hr = H / world_size;
+    // the result pointer is the send buffer; rows are placed by the kernel
+    return lse_combine_impl(fn, partial_outputs, partial_lses, send_buf, nullptr, S, B, H, D, out_stride_s, H * D, D,
+                            lse_stride_s, H, 1, H * D, D, H, 1, dtype, is_lse_base_on_e, 0, cuda_stream, Varlen{}, po);
 }
 
 int32_t dcp_unpack_combine(const void *recv_buf, void *result, float *global_lse, int32_t N, int64_t B, int64_t Hr,

@@ -193,6 +193,12 @@ struct CombineArgs {
     // holds KV of that request iff n * interleave < seq_lens[r].  A shard without
     // KV counts as LSE -inf and its row is not read; a token outside every request
     // combines no shard at all.
+    // PACK_OUT (split layout in, the packed send layout out): unit (b, h) of the H = heads
+    // input heads is written as packed row ((h / pack_hr) * pack_b + b) * pack_hr + h mod
+    // pack_hr, data_w + 1 words per row, the merged fp32 LSE in its last word.
+    int64_t pack_b;
+    int64_t pack_hr;
+    uint64_t pack_hr_magic;  // ceil(2^64 / pack_hr), 0 when pack_hr == 1
     int32_t varlen;
     int32_t num_reqs;
     int32_t interleave;
@@ -345,7 +351,8 @@ __host__ __device__ constexpr size_t combine_smem_bytes(int units_per_warp, int 
 // output chunk c is elements 2q/e.. of sum c and the first ones of sum c+1 (from
 // the next lane, or, for the last chunk, the weighted sum of the tail chunks,
 // formed in phase 1 and reduced over the lane group).
-template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS = 1, bool UNIFORM = false, bool VARLEN = false>
+template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS = 1, bool UNIFORM = false, bool VARLEN = false,
+          bool PACK_OUT = false>
 __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(const CombineArgs a) {
     constexpr int kUnitsPerWarp = 32 / G;
     constexpr int kWarps = kCombineThreads / 32;
@@ -407,6 +414,10 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
             lse_off = b * a.lse_sb + h * a.lse_sh;
             res_off = b * a.res_sb_w + h * a.res_sh_w;
             glse_off = b * a.glse_sb + h * a.glse_sh;
+            if constexpr (PACK_OUT) {
+                const int64_t rank = (int64_t)div_magic((uint64_t)h, a.pack_hr_magic);
+                res_off = ((rank * a.pack_b + b) * a.pack_hr + (h - rank * a.pack_hr)) * (int64_t)(a.data_w + 1);
+            }
             if constexpr (VARLEN) {
                 cp_async_wait<0>();  // lane 0's copies for this task
                 __syncwarp();
@@ -486,7 +497,15 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
         wsum = group_sum<G>(wsum);
         const float denom = fmaxf(wsum, 1e-10f);
         for (int n = j; n < a.N; n += G) sw[n] = sw[n] / denom;
-        if (a.return_lse && valid && j == 0) a.glse[glse_off] = (a.base_e ? logf(wsum) : log2f(wsum)) + m;
+        if constexpr (PACK_OUT) {
+            if (valid && j == 0) {
+                Words<1> lw;
+                lw.w[0] = __float_as_uint((a.base_e ? logf(wsum) : log2f(wsum)) + m);
+                store_words<1>(a.result + res_off + a.data_w, lw);
+            }
+        } else {
+            if (a.return_lse && valid && j == 0) a.glse[glse_off] = (a.base_e ? logf(wsum) : log2f(wsum)) + m;
+        }
 
         // UNIFORM: weighted sum of the shards' tail chunks.  With few shards the lane
         // that owns the row's last chunk sums them itself; otherwise each lane sums its
@@ -594,6 +613,59 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
                     nx.w[3] = 0u;
                     if (act[k] && c[k] == a.chunks - 1) nx = tenc;
                     if (act[k]) store_words<4>(a.result + res_off + 4 * (int64_t)c[k], funnel_words(enc[k], nx, q));
+                }
+            } else if constexpr (PACK_OUT) {
+                // The packed row starts q = res_off mod 4 words past a 16-byte boundary.
+                // Interior: the aligned chunk at row word 4c + 4 - q is words 4 - q.. of
+                // output chunk c and the first q words of chunk c + 1 (from the next lane,
+                // lane 0's next slot for lane G-1).  The row's first 4 - q and last q words
+                // are written one by one, so no store touches a neighbouring row.  Rows that
+                // take more than one pass are written word by word.
+                const int q = (int)(res_off & 3);
+                uint32_t *rowp = a.result + res_off;
+                Words<4> enc[CPL];
+#pragma unroll
+                for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) enc[k].w[e] = T::encode(&acc[k][e * T::kPerWord]);
+                if (a.slots <= CPL) {  // one pass: every chunk of the row is in registers
+#pragma unroll
+                    for (int k = 0; k < CPL; ++k) {
+                        Words<4> send = enc[k];
+                        if (k + 1 < CPL && j == 0) send = enc[k + 1 < CPL ? k + 1 : k];
+                        Words<4> nx;
+#pragma unroll
+                        for (int e = 0; e < 3; ++e) nx.w[e] = __shfl_sync(0xffffffffu, send.w[e], next_lane);
+                        nx.w[3] = 0u;
+                        if (!act[k]) continue;
+                        const int cc = c[k];
+                        if (q == 0) {
+                            store_words<4>(rowp + 4 * cc, enc[k]);
+                            continue;
+                        }
+                        if (cc + 1 < a.chunks) store_words<4>(rowp + 4 * cc + 4 - q, funnel_words(enc[k], nx, 4 - q));
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const bool head = cc == 0 && e < 4 - q;
+                            const bool tail = cc + 1 == a.chunks && e >= 4 - q;
+                            if (head || tail) {
+                                Words<1> wv;
+                                wv.w[0] = enc[k].w[e];
+                                store_words<1>(rowp + 4 * cc + e, wv);
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < CPL; ++k) {
+                        if (!act[k]) continue;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            Words<1> wv;
+                            wv.w[0] = enc[k].w[e];
+                            store_words<1>(rowp + 4 * c[k] + e, wv);
+                        }
+                    }
                 }
             } else {
 #pragma unroll

@@ -12,6 +12,7 @@
  *   dcp_lse_combine          combine of separate output / LSE receive buffers
  *   dcp_lse_combine_strided  the same with any token / head layout
  *   dcp_lse_combine_varlen   the same per request: shards without KV are skipped
+ *   dcp_combine_pack         a producer's split merge written straight into the send buffer
  *   dcp_unpack_combine       combine read straight out of the packed buffer
  *
  * Defining passages (web pages, by title and section):
@@ -200,6 +201,32 @@ int32_t dcp_lse_combine_varlen(const void *outputs, const float *lses, void *res
                                const int32_t *seq_lens, const int32_t *query_start_loc,
                                int32_t num_reqs, int32_t interleave, int32_t dtype,
                                int32_t is_lse_base_on_e, int32_t return_lse, void *cuda_stream);
+
+/*
+ * Combine fused with the pack: the producer's epilogue.  A split-KV (flash-decoding)
+ * producer ends by merging its S partial results over its own KV splits, by the same
+ * [COMBINE] rules; this call does that merge and writes the merged rows straight into the
+ * [A2A] send buffer, so cp_attn_out is never written and dcp_pack never runs.
+ * Equivalent to dcp_lse_combine(..., return_lse = 1) into [B, H, D] + [B, H], then
+ * dcp_pack of those into send_buf, with the same bits.
+ *
+ * partial_outputs  [S, B, H, D] of `dtype`; element (s, b, h, d) at
+ *             s*out_stride_s + (b*H + h)*D + d, out_stride_s >= B*H*D.
+ * partial_lses     [S, B, H] fp32; element (s, b, h) at s*lse_stride_s + b*H + h,
+ *             lse_stride_s >= B*H.
+ * send_buf    [world_size, B, H/world_size, D + P] of `dtype`, contiguous (as written
+ *             by dcp_pack): row (r, b, h) receives the merged row of head r*H/world_size
+ *             + h, then the 4 bytes of its merged fp32 LSE (ln S + m, or log2 S + m).
+ *
+ * Requirements: S in [1, DCP_MAX_SHARDS]; world_size in [1, DCP_MAX_SHARDS]; H %
+ * world_size == 0 (else DCP_ERR_SHAPE); B >= 0; H, D >= 1; D*elemsize a multiple of 16;
+ * partial_outputs and send_buf 16-byte aligned; out_stride_s a multiple of 16/elemsize;
+ * partial_lses 4-byte aligned.
+ */
+int32_t dcp_combine_pack(const void *partial_outputs, const float *partial_lses, void *send_buf,
+                         int32_t S, int64_t B, int64_t H, int64_t D,
+                         int64_t out_stride_s, int64_t lse_stride_s, int32_t world_size,
+                         int32_t dtype, int32_t is_lse_base_on_e, void *cuda_stream);
 
 /*
  * Fused unpack + combine over the packed receive buffer ([A2A], the step

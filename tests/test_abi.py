@@ -203,3 +203,31 @@ def test_varlen_rejections(lib):
     assert _varlen(lib, outputs=A + 8) == MISALIGNED
     assert _varlen(lib, glse=None, ret=1) == INVALID
     assert "dcp_lse_combine_varlen" in dcp.dcp_last_error()
+
+
+def _combine_pack(lib, **kw):
+    a = dict(outputs=A, lses=A, send=A, S=2, B=4, H=16, D=128, ss=None, ls=None, ws=4, dtype=0)
+    a.update(kw)
+    ss = a["ss"] if a["ss"] is not None else a["B"] * a["H"] * a["D"]
+    ls = a["ls"] if a["ls"] is not None else a["B"] * a["H"]
+    return lib.dcp_combine_pack(a["outputs"], a["lses"], a["send"], a["S"], a["B"], a["H"], a["D"], ss, ls, a["ws"],
+                                a["dtype"], 1, None)
+
+
+def test_combine_pack_rejections(lib):
+    assert _combine_pack(lib, B=0) == OK
+    assert _combine_pack(lib, dtype=7) == DTYPE
+    assert _combine_pack(lib, S=0) == INVALID
+    assert _combine_pack(lib, S=65) == INVALID
+    assert _combine_pack(lib, ws=0) == INVALID
+    assert _combine_pack(lib, ws=65) == INVALID
+    assert _combine_pack(lib, H=18, ws=4) == SHAPE
+    assert _combine_pack(lib, D=12) == MISALIGNED
+    assert _combine_pack(lib, ss=4 * 16 * 128 - 8) == INVALID
+    assert _combine_pack(lib, ss=4 * 16 * 128 + 4) == MISALIGNED
+    assert _combine_pack(lib, ls=63) == INVALID
+    assert _combine_pack(lib, send=None) == INVALID
+    assert _combine_pack(lib, send=A + 4) == MISALIGNED
+    assert _combine_pack(lib, outputs=None) == INVALID
+    assert _combine_pack(lib, lses=A + 2) == MISALIGNED
+    assert "dcp_combine_pack" in dcp.dcp_last_error()
