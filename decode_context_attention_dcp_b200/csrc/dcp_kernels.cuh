@@ -512,6 +512,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
         // shards and the group reduces.
         float tacc[kElems];
         if constexpr (PACKED && UNIFORM) {
+            __syncwarp();  // the owning lane reads the weights and tails the other lanes wrote
 #pragma unroll
             for (int e = 0; e < kElems; ++e) tacc[e] = 0.0f;
             const bool few = a.N <= 4;  // the same for the whole warp
