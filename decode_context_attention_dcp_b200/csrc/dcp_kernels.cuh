@@ -128,6 +128,15 @@ __device__ __forceinline__ void cp_async_chunk(void *s, const uint32_t *g) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(s)), "l"(g));
 }
 
+// The 16-byte chunk at word w of a 16-byte aligned buffer into shared memory, copying
+// only the words below `limit` (the rest of the destination is zero-filled, and nothing
+// at or past `limit` is read).  At least one word must lie below `limit`.
+__device__ __forceinline__ void cp_async_chunk_bounded(void *s, const uint32_t *base, int64_t w, int64_t limit) {
+    const int64_t left = limit - w;
+    const uint32_t bytes = left >= 4 ? 16u : (uint32_t)(4 * left);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(s)), "l"(base + w), "r"(bytes));
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
 template <int PENDING>
@@ -324,10 +333,13 @@ __device__ __forceinline__ Words<4> load_chunk_bounded(const uint32_t *base, int
     return r;
 }
 
-// Shared memory of one combine CTA: per warp and per row in flight, the N
-// normalised weights, and (packed layout) the N tail chunks.
-__host__ __device__ constexpr size_t combine_smem_bytes(int units_per_warp, int N, bool packed) {
-    return (size_t)(kCombineThreads / 32) * units_per_warp * N * (sizeof(float) + (packed ? 16 : 0));
+// Shared memory of one combine CTA: per warp and per row in flight, the N normalised
+// weights and what phase 1 reads for N shards: the rows' aligned tail chunks (packed
+// layout), and with `prefetch` two buffers of them (or of the LSE words, split layout),
+// filled one task ahead.
+__host__ __device__ constexpr size_t combine_smem_bytes(int units_per_warp, int N, bool packed, bool prefetch) {
+    return (size_t)(kCombineThreads / 32) * units_per_warp * N *
+           (sizeof(float) + (prefetch ? 2 : 1) * (packed ? 16 : 0) + (prefetch && !packed ? 2 * 4 : 0));
 }
 
 // One warp works on 32/G result rows at a time, G lanes per row; lane j of a row
@@ -352,8 +364,9 @@ __host__ __device__ constexpr size_t combine_smem_bytes(int units_per_warp, int 
 // the next lane, or, for the last chunk, the weighted sum of the tail chunks,
 // formed in phase 1 and reduced over the lane group).
 template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS = 1, bool UNIFORM = false, bool VARLEN = false,
-          bool PACK_OUT = false>
+          bool PACK_OUT = false, bool PREFETCH = false>
 __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(const CombineArgs a) {
+    static_assert(!VARLEN || PREFETCH, "the variable-length combine prefetches its request guesses");
     constexpr int kUnitsPerWarp = 32 / G;
     constexpr int kWarps = kCombineThreads / 32;
     constexpr int kElems = 4 * T::kPerWord;
@@ -365,27 +378,51 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
     const int j = lane % G;
     const int next_lane = (lane & ~(G - 1)) | ((j + 1) & (G - 1));
     const int slot_base = warp * kUnitsPerWarp + ul;
-    uint4 *s_tail = s_dyn + (size_t)slot_base * a.N;  // packed only: [warps * units_per_warp][N]
-    float *sw = reinterpret_cast<float *>(s_dyn + (PACKED ? (size_t)kWarps * kUnitsPerWarp * a.N : 0)) +
-                (size_t)slot_base * a.N;
+    constexpr int kRows = kWarps * kUnitsPerWarp;  // rows in flight per CTA
+    constexpr int kBufs = PREFETCH ? 2 : 1;
+    // packed: tail chunks [kBufs][kRows][N] (uint4); split with PREFETCH: LSE words
+    // [2][kRows][N]; then the weights [kRows][N]
+    uint4 *s_tail_all = s_dyn;
+    uint32_t *s_lse = reinterpret_cast<uint32_t *>(s_dyn);
+    float *sw = reinterpret_cast<float *>(s_dyn) +
+                (size_t)kRows * a.N * (PACKED ? 4 * kBufs : (PREFETCH ? 2 : 0)) + (size_t)slot_base * a.N;
     const int64_t tasks = (a.units + kUnitsPerWarp - 1) / kUnitsPerWarp;
-    // VARLEN: for each row's next token, lane 0 of the row copies qsl[g], qsl[g + 1] and
-    // seq_lens[g] (g = varlen_guess) into shared memory one task ahead (two buffers,
-    // alternating), so the usual case waits on no global read.
-    __shared__ int32_t s_probe[VARLEN ? 2 : 1][VARLEN ? 3 * kWarps * kUnitsPerWarp : 1];
+    // What phase 1 reads for each row's next task -- the LSE words (split layout) or the
+    // rows' aligned tail chunks, which hold the LSE (packed layout) -- is copied into shared
+    // memory one task ahead (two buffers, alternating), so phase 1 waits on no global read.
+    // VARLEN: lane 0 of the row also copies qsl[g], qsl[g + 1] and seq_lens[g]
+    // (g = varlen_guess) of the next token.  One copy group per task.
+    __shared__ int32_t s_probe[VARLEN ? 2 : 1][VARLEN ? 3 * kRows : 1];
     int64_t qsl_end = 0;
     float r_per_token = 0.0f;
     const int64_t full_seq = (int64_t)(a.N - 1) * a.interleave;
     int buf = 0;
-    auto fetch_guess = [&](int64_t t, int into) {
+    auto prefetch = [&](int64_t t, int into) {
         const int64_t uu = t * kUnitsPerWarp + ul;
-        if (j == 0 && uu < a.units && a.num_reqs > 0) {
-            const int64_t bb = (int64_t)div_magic((uint64_t)uu, a.heads_magic);
-            const int g = varlen_guess(bb, a.num_reqs, qsl_end, r_per_token);
-            uint32_t *d = reinterpret_cast<uint32_t *>(&s_probe[into][3 * slot_base]);
-            cp_async_word(d, reinterpret_cast<const uint32_t *>(a.qsl + g));
-            cp_async_word(d + 1, reinterpret_cast<const uint32_t *>(a.qsl + g + 1));
-            cp_async_word(d + 2, reinterpret_cast<const uint32_t *>(a.seq_lens + g));
+        if (uu < a.units) {
+            if constexpr (PACKED) {
+                uint4 *dst = s_tail_all + ((size_t)into * kRows + slot_base) * a.N;
+                const int64_t rw = uu * a.row_pitch_w;  // the row's first word in shard 0
+                for (int n = j; n < a.N; n += G) {
+                    const int64_t wa = ((int64_t)n * a.shard_stride_w + rw) & ~int64_t(3);
+                    cp_async_chunk_bounded(dst + n, a.src, wa + 4 * (int64_t)a.chunks, a.total_w);
+                }
+            } else {
+                uint32_t *dst = s_lse + ((size_t)into * kRows + slot_base) * a.N;
+                const int64_t bb = (int64_t)div_magic((uint64_t)uu, a.heads_magic);
+                const int64_t lo = bb * a.lse_sb + (uu - bb * a.heads) * a.lse_sh;
+                const uint32_t *lses = reinterpret_cast<const uint32_t *>(a.lses);
+                for (int n = j; n < a.N; n += G) cp_async_word(dst + n, lses + n * a.lse_stride_n + lo);
+                if constexpr (VARLEN) {
+                    if (j == 0 && a.num_reqs > 0) {
+                        const int g = varlen_guess(bb, a.num_reqs, qsl_end, r_per_token);
+                        uint32_t *d = reinterpret_cast<uint32_t *>(&s_probe[into][3 * slot_base]);
+                        cp_async_word(d, reinterpret_cast<const uint32_t *>(a.qsl + g));
+                        cp_async_word(d + 1, reinterpret_cast<const uint32_t *>(a.qsl + g + 1));
+                        cp_async_word(d + 2, reinterpret_cast<const uint32_t *>(a.seq_lens + g));
+                    }
+                }
+            }
         }
         cp_async_commit();
     };
@@ -394,19 +431,18 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
             qsl_end = __ldg(a.qsl + a.num_reqs);
             if (qsl_end > 0) r_per_token = (float)a.num_reqs / (float)qsl_end;
         }
-        fetch_guess((int64_t)blockIdx.x * kWarps + warp, 0);
     }
+    if constexpr (PREFETCH) prefetch((int64_t)blockIdx.x * kWarps + warp, 0);
 
     for (int64_t task = (int64_t)blockIdx.x * kWarps + warp; task < tasks; task += (int64_t)gridDim.x * kWarps) {
         const int64_t u = task * kUnitsPerWarp + ul;
         const bool valid = u < a.units;
-        int64_t row, lse_off, res_off, glse_off;
+        int64_t row, res_off, glse_off, lse_off = 0;
         int nk = a.N;  // shards [0, nk) are read; the rest weigh 0
         if constexpr (PACKED) {
             row = u * a.row_pitch_w;
             res_off = u * a.data_w;
             glse_off = u;
-            lse_off = 0;
         } else {
             const int64_t b = (int64_t)div_magic((uint64_t)u, a.heads_magic);
             const int64_t h = u - b * a.heads;
@@ -419,7 +455,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
                 res_off = ((rank * a.pack_b + b) * a.pack_hr + (h - rank * a.pack_hr)) * (int64_t)(a.data_w + 1);
             }
             if constexpr (VARLEN) {
-                cp_async_wait<0>();  // lane 0's copies for this task
+                cp_async_wait<0>();  // this task's prefetch (lane 0's guess copies among them)
                 __syncwarp();
                 const int32_t *pr = &s_probe[buf][3 * slot_base];
                 nk = varlen_shards<G>(a, b, valid, j, qsl_end, r_per_token, full_seq, pr[0], pr[1], pr[2]);
@@ -458,26 +494,35 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
 
         set_pass(0);
         issue(0);
-        if constexpr (VARLEN) {
-            buf ^= 1;
-            fetch_guess(task + (int64_t)gridDim.x * kWarps, buf);
-        }
+        if constexpr (PREFETCH) prefetch(task + (int64_t)gridDim.x * kWarps, buf ^ 1);
+        uint4 *s_tail = s_tail_all + ((size_t)buf * kRows + slot_base) * a.N;  // packed: this task's tails
 
         // ---- phase 1: weights of the N shards --------------------------------
+        if constexpr (PREFETCH) cp_async_wait<1>();  // this task's copies (each lane reads the ones it made)
+        const uint32_t *lse_now = s_lse + ((size_t)buf * kRows + slot_base) * a.N;
         float lmax = -INFINITY;
         for (int n = j; n < a.N; n += G) {
             float l = -INFINITY;
             if (valid && n < nk) {
                 uint32_t bits;
+                const int64_t w0 = (int64_t)n * a.shard_stride_w + row;
                 if constexpr (PACKED) {
-                    const int64_t w0 = (int64_t)n * a.shard_stride_w + row;
-                    const int64_t wa = w0 & ~int64_t(3);
-                    const Words<4> t = load_chunk_bounded(a.src, wa + 4 * (int64_t)a.chunks, a.total_w);
-                    s_tail[n] = make_uint4(t.w[0], t.w[1], t.w[2], t.w[3]);
+                    uint4 t;
+                    if constexpr (PREFETCH) {
+                        t = s_tail[n];
+                    } else {
+                        const Words<4> v = load_chunk_bounded(a.src, (w0 & ~int64_t(3)) + 4 * (int64_t)a.chunks, a.total_w);
+                        t = make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]);
+                        s_tail[n] = t;
+                    }
                     const int q = (int)(w0 & 3);
-                    bits = q == 0 ? t.w[0] : q == 1 ? t.w[1] : q == 2 ? t.w[2] : t.w[3];
+                    bits = q == 0 ? t.x : q == 1 ? t.y : q == 2 ? t.z : t.w;
                 } else {
-                    bits = load_word(reinterpret_cast<const uint32_t *>(a.lses) + n * a.lse_stride_n + lse_off);
+                    if constexpr (PREFETCH) {
+                        bits = lse_now[n];
+                    } else {
+                        bits = load_word(reinterpret_cast<const uint32_t *>(a.lses) + n * a.lse_stride_n + lse_off);
+                    }
                 }
                 l = sanitize_lse(bits);
             }
@@ -510,9 +555,9 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
         // UNIFORM: weighted sum of the shards' tail chunks.  With few shards the lane
         // that owns the row's last chunk sums them itself; otherwise each lane sums its
         // shards and the group reduces.
+        __syncwarp();  // lanes read the weights and tail chunks other lanes wrote
         float tacc[kElems];
         if constexpr (PACKED && UNIFORM) {
-            __syncwarp();  // the owning lane reads the weights and tails the other lanes wrote
 #pragma unroll
             for (int e = 0; e < kElems; ++e) tacc[e] = 0.0f;
             const bool few = a.N <= 4;  // the same for the whole warp
@@ -681,7 +726,9 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
             }
         }
         __syncwarp();
+        if constexpr (PREFETCH) buf ^= 1;
     }
+    if constexpr (PREFETCH) cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
