@@ -14,7 +14,7 @@ Low-level calls (same names as the C ABI, caller-allocated outputs):
     dcp_lse_combine_varlen(outputs, lses, result, seq_lens, query_start_loc, ...)
     dcp_combine_pack(partial_outputs, partial_lses, send_buf, world_size, ...)
     dcp_unpack_combine(recv_buf, result, global_lse=None, ...)
-    dcp_lse_pack_dim(dtype), dcp_last_error()
+    dcp_lse_pack_dim(dtype), dcp_last_error(), dcp_wait_timeouts(reset=False)
 
 Allocating helpers with the pages' argument conventions:
     lse_weighted_combine(outputs, lses, return_lse=False, is_lse_base_on_e=True)
@@ -35,7 +35,7 @@ from . import _build
 
 __all__ = [
     "DCPError", "library", "dcp_lse_pack_dim", "dcp_pack", "dcp_lse_combine", "dcp_lse_combine_varlen",
-    "dcp_combine_pack", "dcp_unpack_combine", "combine_pack", "dcp_last_error", "dcp_version", "lse_weighted_combine", "lse_weighted_combine_varlen",
+    "dcp_combine_pack", "dcp_unpack_combine", "combine_pack", "dcp_last_error", "dcp_version", "dcp_wait_timeouts", "lse_weighted_combine", "lse_weighted_combine_varlen",
     "merge_dcp_outputs", "pack", "unpack_combine",
     "DTYPE_CODES",
 ]
@@ -87,6 +87,8 @@ def library() -> ctypes.CDLL:
                 lib.dcp_unpack_combine.restype = _i32
                 lib.dcp_last_error.argtypes = []
                 lib.dcp_last_error.restype = ctypes.c_char_p
+                lib.dcp_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint64), _i32]
+                lib.dcp_wait_timeouts.restype = _i32
                 lib.dcp_version.argtypes = []
                 lib.dcp_version.restype = _i32
                 _lib = lib
@@ -95,6 +97,14 @@ def library() -> ctypes.CDLL:
 
 def dcp_last_error() -> str:
     return library().dcp_last_error().decode()
+
+
+def dcp_wait_timeouts(reset: bool = False) -> int:
+    """Waits that timed out on the current device since the last reset (synchronises the
+    device).  Nonzero means some dcp_pack result is incomplete."""
+    c = ctypes.c_uint64(0)
+    _check(library().dcp_wait_timeouts(ctypes.byref(c), int(bool(reset))))
+    return int(c.value)
 
 
 def dcp_version() -> int:

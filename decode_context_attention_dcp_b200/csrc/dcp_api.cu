@@ -249,6 +249,19 @@ extern "C" {
 
 int32_t dcp_version(void) { return 10000; }
 
+int32_t dcp_wait_timeouts(uint64_t *count, int32_t reset) {
+    if (!count) return fail(DCP_ERR_INVALID_ARG, "dcp_wait_timeouts: count is null");
+    unsigned long long v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, dcp::g_wait_timeouts, sizeof(v));
+    if (e == cudaSuccess && reset) {
+        const unsigned long long zero = 0;
+        e = cudaMemcpyToSymbol(dcp::g_wait_timeouts, &zero, sizeof(zero));
+    }
+    if (e != cudaSuccess) return fail(DCP_ERR_CUDA, "dcp_wait_timeouts: %s", cudaGetErrorString(e));
+    *count = v;
+    return ok();
+}
+
 const char *dcp_last_error(void) { return g_error; }
 
 int32_t dcp_lse_pack_dim(int32_t dtype) {

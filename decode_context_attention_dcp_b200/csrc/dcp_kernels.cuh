@@ -144,6 +144,64 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(PENDING) : "memory");
 }
 
+// mbarrier and bulk-copy helpers (shared-memory barrier objects, 8 bytes each).
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// Makes barrier initialisation visible to the copy engine.
+__device__ __forceinline__ void mbar_fence_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+// Orders this thread's earlier shared-memory accesses before its later bulk copies.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Waits that time out: counted here, read (and cleared) by the host with dcp_wait_timeouts.
+__device__ unsigned long long g_wait_timeouts = 0;
+
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // one second
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits for the barrier's phase with the given parity; false when a second passes (or the
+// iteration cap is reached) first.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t spin = 0; spin < (1u << 26); ++spin) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitLimitNs) break;
+    }
+    return false;
+}
+
+// Global -> shared bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned),
+// completing as transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
 // n / d for n < 2^32 and d <= 2^32, with magic = ceil(2^64 / d) (0 meaning d == 1).
 __device__ __forceinline__ uint64_t div_magic(uint64_t n, uint64_t magic) {
     return magic ? __umul64hi(n, magic) : n;
@@ -780,6 +838,8 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
     uint32_t *s_stage = reinterpret_cast<uint32_t *>(s_stage_v4);
     __shared__ int64_t s_row_src[kPackStages][kPackMaxTileRows];  // word offset of each source row
     __shared__ int64_t s_row_lse[kPackStages][kPackMaxTileRows];  // index of each row's LSE
+    __shared__ uint64_t s_full[kPackStages];                      // a stage's rows have landed
+    __shared__ int s_abort;                                       // a wait timed out
     const int tid = threadIdx.x;
     const int64_t tiles = (a.rows + a.tile_rows - 1) / a.tile_rows;
     const int64_t my_tiles = tiles > blockIdx.x ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
@@ -820,18 +880,29 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
     const int lane = tid & 31;
     const int sub = lane % lpr;
     const int row_first = (tid >> 5) * rpw + lane / lpr;
+    // each source row is one bulk copy (16-byte aligned, a multiple of 16 bytes) that
+    // completes on the stage's barrier; the LSE words are 4-byte cp.async copies
+    const uint32_t row_bytes = (uint32_t)data_w * 4u;
     auto issue = [&](int64_t k) {
         const int nrows = tile_rows_of(k);
         const int slot = (int)(k % kPackStages);
         uint32_t *stage = s_stage + slot * stage_w;
-        for (int r = row_first; r < nrows; r += kPackThreads / lpr) {
-            const uint32_t *srow = src + s_row_src[slot][r];
-            uint32_t *drow = stage + r * data_w;
-            for (int c = sub; c < chunks; c += lpr) cp_async_chunk(drow + 4 * c, srow + 4 * c);
-            if (sub == 0) cp_async_word(stage + lse_base + r, lse + s_row_lse[slot][r]);
+        if (tid == 0) mbar_arrive_expect_tx(&s_full[slot], (uint32_t)nrows * row_bytes);
+        for (int r = tid; r < nrows; r += kPackThreads) {
+            fence_proxy_async();
+            bulk_copy_g2s(stage + r * data_w, src + s_row_src[slot][r], row_bytes, &s_full[slot]);
+            cp_async_word(stage + lse_base + r, lse + s_row_lse[slot][r]);
         }
     };
+    (void)lpr;
+    (void)sub;
+    (void)row_first;
 
+    if (tid == 0) {
+        for (int st = 0; st < kPackStages; ++st) mbar_init(&s_full[st], 1);
+        mbar_fence_init();
+        s_abort = 0;
+    }
     for (int64_t k = 0; k < kPackStages && k < my_tiles; ++k) fill_table(k);
     __syncthreads();
 #pragma unroll
@@ -846,8 +917,21 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
         // tile k's table slot was last read when tile k's copies were issued: fill it
         // for tile k + kPackStages while the copies are in flight
         if (k + kPackStages < my_tiles) fill_table(k + kPackStages);
-        cp_async_wait<kPackStages - 1>();  // this thread's copies of tile k have landed
+        cp_async_wait<kPackStages - 1>();  // this thread's LSE copies of tile k have landed
+        // the rows of tile k; a wait that times out is counted, and the CTA waits once more
+        // (bounded) for the copies it has in flight, then stops
+        uint64_t *bar = &s_full[(int)(k % kPackStages)];
+        const uint32_t parity = (uint32_t)((k / kPackStages) & 1);
+        if (!mbar_wait_bounded(bar, parity)) {
+            atomicAdd(&g_wait_timeouts, 1ull);
+            s_abort = 1;
+        }
         __syncthreads();                   // ... and everyone else's (and the table)
+        if (s_abort) {
+            mbar_wait_bounded(bar, parity);
+            cp_async_wait<0>();
+            return;
+        }
 
         const int64_t i0 = (blockIdx.x + k * gridDim.x) * tile_rows;
         const int nrows = tile_rows_of(k);

@@ -42,7 +42,7 @@
  * Conventions shared by every entry point:
  *   - All buffer pointers are DEVICE pointers on the device that is current on
  *     the calling thread; the caller owns every buffer.  The library allocates
- *     nothing and keeps no state besides a per-thread error message.
+ *     nothing.
  *   - Calls are asynchronous on `cuda_stream` (a cudaStream_t; NULL = the
  *     legacy default stream) and never synchronise.  Inputs must stay valid
  *     and outputs untouched until the stream reaches the call.
@@ -52,7 +52,8 @@
  *     dcp_status is returned and nothing is launched.  dcp_last_error() then
  *     describes the problem.  A failed launch returns DCP_ERR_CUDA.
  *   - B == 0 is a valid no-op.
- *   - Thread-safe: no global mutable state (the error text is thread-local).
+ *   - Thread-safe: no global mutable state besides the per-thread error text and the
+ *     device's count of timed-out waits (dcp_wait_timeouts).
  */
 #ifndef DCP_COMBINE_H
 #define DCP_COMBINE_H
@@ -246,6 +247,16 @@ int32_t dcp_unpack_combine(const void *recv_buf, void *result, float *global_lse
                            int32_t N, int64_t B, int64_t Hr, int64_t D, int64_t stride_n,
                            int32_t dtype, int32_t is_lse_base_on_e, int32_t return_lse,
                            void *cuda_stream);
+
+/*
+ * Waits that timed out on the current device since the last reset.  dcp_pack waits for
+ * its bulk copies with a limit of about one second per wait; a wait that runs out is
+ * counted here and the CTA stops, so the send buffer of that call is incomplete.  A
+ * nonzero count therefore means a result is invalid (it never happens when the copies
+ * work).  Synchronises the device (the counter is read from device memory); with reset
+ * != 0 the counter is cleared afterwards.  Returns DCP_ERR_CUDA if the read fails.
+ */
+int32_t dcp_wait_timeouts(uint64_t *count, int32_t reset);
 
 /* Text of the last non-OK status returned on the calling thread ("" if none). */
 const char *dcp_last_error(void);

@@ -449,3 +449,11 @@ def test_cuda_graph_replay(o):
         ry, rg = o.unpack_combine(ref_send, orc.BF16, D, return_lse=True)
         assert_out_close(y, ry, f"graph replay seed {seed}")
         assert_lse_close(g, rg, f"graph replay seed {seed} lse")
+
+
+def test_no_wait_timed_out():
+    """Every bulk-copy wait of the kernels run so far completed within its limit (a timeout
+    would mean an incomplete send buffer)."""
+    torch.cuda.synchronize()
+    assert dcp.dcp_wait_timeouts() == 0
+    assert dcp.dcp_wait_timeouts(reset=True) == 0
