@@ -195,6 +195,9 @@ int32_t dispatch_combine(dcp::CombineArgs a, cudaStream_t stream) {
     const bool uniform = PACKED && (a.N == 1 || a.shard_stride_w % 4 == 0) && chunks <= 4 * 32;
     int cpl_target = a.N >= 8 ? 1 : a.N >= 4 ? 2 : 4;
     if (PACKED && !uniform && cpl_target < 2) cpl_target = 2;
+    // split layout, 8-15 shards, rows of at most 256 bytes: two chunk slots per lane (four
+    // rows per warp) measured 3-6% faster than one; packed rows lose with more slots
+    if (!PACKED && a.N >= 8 && a.N < 16 && chunks <= 16) cpl_target = 2;
     const int per_lane = (chunks + cpl_target - 1) / cpl_target;
     int G = 4;
     while (G < per_lane && G < 32) G *= 2;
