@@ -457,3 +457,34 @@ def test_no_wait_timed_out():
     torch.cuda.synchronize()
     assert dcp.dcp_wait_timeouts() == 0
     assert dcp.dcp_wait_timeouts(reset=True) == 0
+
+
+PACK_EDGE = [  # B, H, D, world_size, dtype
+    (3, 4, 8192, 2, "bf16"), (2, 3, 8192, 3, "fp32"), (5, 6, 4096, 3, "fp32"), (9, 5, 2048, 5, "bf16"),
+    (301, 7, 8, 7, "bf16"), (97, 8, 4, 2, "fp32"), (130, 16, 128, 16, "fp16"), (64, 64, 64, 1, "bf16"),
+    (1, 1, 16, 1, "fp16"), (33, 12, 520, 4, "bf16"), (3, 2, 1032, 2, "fp32")]
+
+
+@pytest.mark.parametrize("B,H,D,ws,dtype", PACK_EDGE)
+def test_pack_edge_shapes(o, B, H, D, ws, dtype):
+    """Bit-exact pack for wide rows (one bulk copy of up to 32 KiB, one row per tile), 16-byte
+    rows, many ragged tiles, world sizes 1 .. H, strided inputs and NaN payloads, with guard
+    bands around the send buffer."""
+    dt = wl.torch_dtype(dtype)
+    gen = torch.Generator().manual_seed(B * 131 + H * 17 + D)
+    big = torch.randn(B, H + 1, D + 8, generator=gen).to(dt)
+    lse_big = torch.randn(B, H + 3, generator=gen)
+    lse_big.view(torch.int32)[0, 0] = 0x7FC0ABCD         # NaN payload must survive
+    if H > 1:
+        lse_big[0, 1] = float("-inf")
+    out, lse = big[:, 1:, :D], lse_big[:, :H]
+    out_d = big.cuda()[:, 1:, :D]                        # strides (H+1)*(D+8), D+8, 1 on the device
+    lse_d = lse_big.cuda()[:, :H]                        # row stride H+3
+    assert out_d.stride() == ((H + 1) * (D + 8), D + 8, 1) and lse_d.stride() == (H + 3, 1)
+    P = dcp.dcp_lse_pack_dim(dt)
+    send = Guarded((ws, B, H // ws, D + P), dt)
+    dcp.dcp_pack(out_d, lse_d, send.tensor, ws)
+    send.check()
+    ref = o.pack(raw(out.contiguous()), raw(lse.contiguous()), ws, ORACLE_CODE[dt])
+    assert np.array_equal(bits(send.tensor.cpu()), bits(ref))
+    assert dcp.dcp_wait_timeouts() == 0
