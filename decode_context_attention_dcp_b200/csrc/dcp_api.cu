@@ -527,8 +527,6 @@ int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_b
     a.per_rank_magic = magic64((uint64_t)(B * a.Hr));
     a.hr_magic = magic64((uint64_t)a.Hr);
     a.pitch_magic = (uint32_t)(((uint64_t(1) << 32) + (uint64_t)a.row_pitch_w - 1) / (uint64_t)a.row_pitch_w);
-    const uint64_t chunks = (uint64_t)a.data_w / 4;
-    a.lanes_per_row = chunks >= 32 ? 32 : chunks >= 16 ? 16 : chunks >= 8 ? 8 : 4;
     const size_t smem = (size_t)dcp::kPackStages * a.stage_w * 4;
     if (!pack_smem_reserved()) return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory for the pack kernel", fn);
     const int per_sm = pack_resident_ctas(smem);

@@ -808,12 +808,80 @@ struct PackArgs {
     uint64_t per_rank_magic;  // ceil(2^64 / (B * Hr)), 0 when B * Hr == 1
     uint64_t hr_magic;        // ceil(2^64 / Hr), 0 when Hr == 1
     uint32_t pitch_magic;     // ceil(2^32 / row_pitch_w): t / row_pitch_w == umulhi(t, magic) when t * row_pitch_w < 2^32
-    int32_t lanes_per_row;    // lanes that copy one source row: 4, 8, 16 or 32
     int32_t data_w;           // words of data per row (a multiple of 4)
     int32_t row_pitch_w;      // data_w + 1: words per packed row
     int32_t tile_rows;        // packed rows per tile
     int32_t stage_w;          // words per shared-memory stage (a multiple of 4)
 };
+
+// Stores one landed tile: packed rows [i0, i0 + nrows) form the send range of words
+// [d0, d0 + nrows * pitch).  The stage holds the tile's source rows one after another
+// (data_w words each), then their LSE words from word lse_base.  Packed word t of the
+// range is row r = t / pitch, word kk = t mod pitch, i.e. stage word t - r when kk < data_w,
+// else LSE r.  Pass 1 writes every whole 16-byte chunk that lies inside one row's data as
+// two aligned 16-byte shared loads and a word funnel.  Pass 2 writes, one thread per row,
+// the chunk that holds the row's LSE word (rows are >= 5 words, so a chunk holds at most
+// one LSE).  The partial chunks at the two ends of the range use 4-byte stores.  Threads
+// tid = 0 .. nthreads - 1 (nthreads >= 8) share the work.
+__device__ __forceinline__ void pack_store_tile(const uint32_t *stage, uint32_t *dst, int64_t d0, int nrows, int data_w,
+                                                int pitch, int lse_base, uint32_t pitch_magic, int tid, int nthreads) {
+    const int len = nrows * pitch;
+    const uint4 *stage_v4 = reinterpret_cast<const uint4 *>(stage);
+    auto word_of = [&](int r, int kk) -> uint32_t {  // word kk of packed row r of the tile
+        return kk < data_w ? stage[r * data_w + kk] : stage[lse_base + r];
+    };
+    const int lead = (int)((4 - (d0 & 3)) & 3);  // words before the first 16-byte boundary
+    const int full = (len - lead) >> 2;           // whole 16-byte chunks of the range
+    uint32_t *dst_full = dst + d0 + lead;         // 16-byte aligned; chunk g = words lead+4g .. +3
+
+    // pass 1: chunks inside one row's data
+    for (int g = tid; g < full; g += nthreads) {
+        const int t0 = lead + 4 * g;
+        const int r = (int)__umulhi((uint32_t)t0, pitch_magic);
+        const int kk = t0 - r * pitch;
+        if (kk + 3 < data_w) {
+            const int base = t0 - r;  // stage word of packed word t0
+            const uint4 lo4 = stage_v4[base >> 2];
+            const uint4 hi4 = stage_v4[(base >> 2) + 1];
+            Words<4> lo, hi;
+            lo.w[0] = lo4.x; lo.w[1] = lo4.y; lo.w[2] = lo4.z; lo.w[3] = lo4.w;
+            hi.w[0] = hi4.x; hi.w[1] = hi4.y; hi.w[2] = hi4.z; hi.w[3] = hi4.w;
+            store_words<4>(dst_full + 4 * g, funnel_words(lo, hi, base & 3));
+        }
+    }
+    // pass 2: the chunk holding each row's LSE word
+    for (int r = tid; r < nrows; r += nthreads) {
+        const int t_row = r * pitch;
+        const int t_lse = t_row + data_w;
+        const int g = (t_lse - lead) >> 2;
+        if (t_lse >= lead && g < full) {
+            Words<4> o;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int kk = lead + 4 * g + e - t_row;
+                o.w[e] = kk < pitch ? word_of(r, kk) : word_of(r + 1, kk - pitch);
+            }
+            store_words<4>(dst_full + 4 * g, o);
+        }
+    }
+    // the partial chunks at the two ends of the range (a range has >= 5 words)
+    auto word_at = [&](int t) -> uint32_t {
+        const int r = (int)__umulhi((uint32_t)t, pitch_magic);
+        return word_of(r, t - r * pitch);
+    };
+    if (tid < lead) {
+        Words<1> o;
+        o.w[0] = word_at(tid);
+        store_words<1>(dst + d0 + tid, o);
+    } else if (tid >= 4 && tid < 8) {
+        const int t = lead + 4 * full + (tid - 4);
+        if (t < len) {
+            Words<1> o;
+            o.w[0] = word_at(t);
+            store_words<1>(dst + d0 + t, o);
+        }
+    }
+}
 
 // A CTA packs tiles of `tile_rows` consecutive packed rows (one contiguous word
 // range of the send buffer), kPackStages tiles in flight.
@@ -848,7 +916,6 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
     const int pitch = a.row_pitch_w;
     const int stage_w = a.stage_w;
     const int lse_base = tile_rows * data_w;  // LSE words follow the rows in a stage
-    const int chunks = data_w >> 2;
     const uint32_t pitch_magic = a.pitch_magic;
     const uint32_t *__restrict__ src = a.src;
     const uint32_t *__restrict__ lse = a.lse;
@@ -873,13 +940,6 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
             s_row_lse[slot][r] = (int64_t)b * a.lse_stride_b + (int64_t)head;
         }
     };
-    // copies of this CTA's k-th tile into stage k % kPackStages: lpr lanes per
-    // source row, consecutive lanes on consecutive 16-byte chunks
-    const int lpr = a.lanes_per_row;
-    const int rpw = 32 / lpr;  // rows per warp at a time
-    const int lane = tid & 31;
-    const int sub = lane % lpr;
-    const int row_first = (tid >> 5) * rpw + lane / lpr;
     // each source row is one bulk copy (16-byte aligned, a multiple of 16 bytes) that
     // completes on the stage's barrier; the LSE words are 4-byte cp.async copies
     const uint32_t row_bytes = (uint32_t)data_w * 4u;
@@ -894,9 +954,6 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
             cp_async_word(stage + lse_base + r, lse + s_row_lse[slot][r]);
         }
     };
-    (void)lpr;
-    (void)sub;
-    (void)row_first;
 
     if (tid == 0) {
         for (int st = 0; st < kPackStages; ++st) mbar_init(&s_full[st], 1);
@@ -934,65 +991,8 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
         }
 
         const int64_t i0 = (blockIdx.x + k * gridDim.x) * tile_rows;
-        const int nrows = tile_rows_of(k);
-        const int64_t d0 = i0 * pitch;  // first send word of the tile
-        const int len = nrows * pitch;
-        const uint32_t *stage = s_stage + (int)(k % kPackStages) * stage_w;
-        const uint4 *stage_v4 = reinterpret_cast<const uint4 *>(stage);
-        auto word_of = [&](int r, int kk) -> uint32_t {  // word kk of packed row r of the tile
-            return kk < data_w ? stage[r * data_w + kk] : stage[lse_base + r];
-        };
-        const int lead = (int)((4 - (d0 & 3)) & 3);  // words before the first 16-byte boundary
-        const int full = (len - lead) >> 2;           // whole 16-byte chunks of the range
-        uint32_t *dst_full = a.dst + d0 + lead;       // 16-byte aligned; chunk g = words lead+4g .. +3
-
-        // pass 1: chunks inside one row's data
-        for (int g = tid; g < full; g += kPackThreads) {
-            const int t0 = lead + 4 * g;
-            const int r = (int)__umulhi((uint32_t)t0, pitch_magic);
-            const int kk = t0 - r * pitch;
-            if (kk + 3 < data_w) {
-                const int base = t0 - r;  // stage word of packed word t0
-                const uint4 lo4 = stage_v4[base >> 2];
-                const uint4 hi4 = stage_v4[(base >> 2) + 1];
-                Words<4> lo, hi;
-                lo.w[0] = lo4.x; lo.w[1] = lo4.y; lo.w[2] = lo4.z; lo.w[3] = lo4.w;
-                hi.w[0] = hi4.x; hi.w[1] = hi4.y; hi.w[2] = hi4.z; hi.w[3] = hi4.w;
-                store_words<4>(dst_full + 4 * g, funnel_words(lo, hi, base & 3));
-            }
-        }
-        // pass 2: the chunk holding each row's LSE word
-        for (int r = tid; r < nrows; r += kPackThreads) {
-            const int t_row = r * pitch;
-            const int t_lse = t_row + data_w;
-            const int g = (t_lse - lead) >> 2;
-            if (t_lse >= lead && g < full) {
-                Words<4> o;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int kk = lead + 4 * g + e - t_row;
-                    o.w[e] = kk < pitch ? word_of(r, kk) : word_of(r + 1, kk - pitch);
-                }
-                store_words<4>(dst_full + 4 * g, o);
-            }
-        }
-        // the partial chunks at the two ends of the range (a range has >= 5 words)
-        auto word_at = [&](int t) -> uint32_t {
-            const int r = (int)__umulhi((uint32_t)t, pitch_magic);
-            return word_of(r, t - r * pitch);
-        };
-        if (tid < lead) {
-            Words<1> o;
-            o.w[0] = word_at(tid);
-            store_words<1>(a.dst + d0 + tid, o);
-        } else if (tid >= 4 && tid < 8) {
-            const int t = lead + 4 * full + (tid - 4);
-            if (t < len) {
-                Words<1> o;
-                o.w[0] = word_at(t);
-                store_words<1>(a.dst + d0 + t, o);
-            }
-        }
+        pack_store_tile(s_stage + (int)(k % kPackStages) * stage_w, a.dst, i0 * pitch, tile_rows_of(k), data_w, pitch,
+                        lse_base, pitch_magic, tid, kPackThreads);
         __syncthreads();  // stage k % kPackStages is free for tile k + kPackStages
     }
     cp_async_wait<0>();
