@@ -113,7 +113,7 @@ def load_peak() -> tuple[float, str]:
 def load_traffic(kernel: str, workload: str) -> float | None:
     """DRAM bytes per launch (read + write) from the committed ncu summary, if it was taken on the
     current kernel sources.  Table rows: | kernel | workload | digest | dram_read | dram_write | ..."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    path = os.path.join(ROOT, "profiles", "dram_traffic_pack_unpack_combine_sweep_N16_B16384_D512.md")
     if not os.path.exists(path):
         return None
     digest = kernel_digest()
