@@ -22,6 +22,7 @@ from __future__ import annotations
 import argparse
 import datetime
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -90,13 +91,17 @@ def barrier(device=None) -> None:
 
 # ---- measurement side data -----------------------------------------------------------------
 def kernel_digest() -> str:
-    """Hash of the kernel sources: ncu counters are reported only for the code they were taken on."""
+    """Hash of the kernel sources' code (comments and whitespace removed): ncu counters are
+    reported only for the code they were taken on."""
     h = hashlib.sha256()
     for sub in ("decode_context_attention_dcp_b200/csrc", "include"):
         d = os.path.join(ROOT, sub)
         for name in sorted(os.listdir(d)):
-            with open(os.path.join(d, name), "rb") as fh:
-                h.update(name.encode() + b"\0" + fh.read())
+            with open(os.path.join(d, name), encoding="utf-8") as fh:
+                text = fh.read()
+            text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+            text = re.sub(r"//[^\n]*", " ", text)
+            h.update(name.encode() + b"\0" + " ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

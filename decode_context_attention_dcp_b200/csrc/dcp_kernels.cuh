@@ -1,11 +1,14 @@
 // dcp_kernels.cuh -- sm_100a kernels of the DCP LSE-weighted combine.
 //
-// Three memory-bound kernels (no tensor cores: the combine is a weighted sum
-// over N shards, ~1 FMA per 2 bytes moved):
+// Memory-bound kernels (no tensor cores: the combine is a weighted sum over N
+// shards, ~1 FMA per 2 bytes moved):
 //
-//   combine_kernel<..., PACKED=false>  combine of split receive buffers
+//   combine_kernel<..., PACKED=false>  combine of split receive buffers (any strides)
+//     VARLEN=true                      ... per request: shards without KV are not read
+//     PACK_OUT=true                    ... written as packed send rows (split merge + pack)
 //   combine_kernel<..., PACKED=true>   fused unpack + combine of the packed buffer
-//   pack_kernel                         output rows + fp32 LSE -> packed rows
+//     PREFETCH=true (either layout)    phase 1's reads copied one task ahead
+//   pack_kernel                         output rows + fp32 LSE -> packed rows (bulk copies)
 //
 // The combine follows vLLM API docs, vllm.v1.attention.ops.dcp_alltoall,
 // _lse_weighted_combine; the packed layout [N, B, H/N, D + P] follows the same
@@ -404,12 +407,17 @@ __host__ __device__ constexpr size_t combine_smem_bytes(int units_per_warp, int 
 // owns its 16-byte chunks j, j+G, j+2G, ... (slots), CPL slots per pass.
 //   1. The loads of the first NB shards' chunks are issued.
 //   2. Phase 1 (weights): lane j takes shards j, j+G, ...; it reads each LSE
-//      (split: from the LSE array; packed: from the row's tail chunk, which it
-//      also keeps in shared memory), sanitises it by exponent bits, and the G
-//      lanes reduce max and sum with xor-shuffles.  The normalised weights go
-//      to shared memory; lane 0 writes the global LSE.
+//      (split: from the LSE array; packed: from the row's tail chunk, which is
+//      kept in shared memory; with PREFETCH both were copied there while the
+//      previous task ran), sanitises it by exponent bits, and the G lanes
+//      reduce max and sum with xor-shuffles.  The normalised weights go to
+//      shared memory; lane 0 writes the global LSE (PACK_OUT: into the packed
+//      row's last word).
 //   3. Phase 2 (weighted sum): fp32 FMAs over all N shards, NB shards' loads
-//      in flight at a time, then one rounding and a 16-byte store per chunk.
+//      in flight at a time, then one rounding and a 16-byte store per chunk
+//      (PACK_OUT: realigned to the packed row, see below).
+// VARLEN: before step 1 the row's lanes find the number of shards holding KV
+// (varlen_shards); loads and LSE reads of the other shards are skipped.
 // Packed rows are 2D+4 bytes, so a row starts q = 0..3 words past a 16-byte
 // boundary.  Lanes load aligned chunks; output chunk c is the 4 words at offset
 // q of aligned chunks c and c+1, and aligned chunk c+1 comes from the next lane
