@@ -9,6 +9,7 @@ statically, so it does not depend on which libcudart the host process loaded.
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -21,7 +22,8 @@ INCLUDE = os.path.join(ROOT, "include")
 CSRC = os.path.join(PKG, "csrc")
 LIBRARY = os.path.join(PKG, "libdcpcombine.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "-shared", "--cudart", "static"]
+COMPILE_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2"]
+LINK_FLAGS = ["-shared", "--cudart", "static"]
 
 
 def nvcc() -> str:
@@ -46,25 +48,39 @@ def stale(lib: str = LIBRARY) -> bool:
     return any(os.path.getmtime(p) > t for p in inputs())
 
 
+def _run(cmd: list[str]) -> None:
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu under csrc/ into one shared library (atomic replace)."""
+    """Compile every .cu under csrc/ (in parallel, one object each) and link them into one
+    shared library (atomic replace)."""
     if not force and not stale():
         return LIBRARY
     fd, tmp = tempfile.mkstemp(suffix=".so", dir=PKG)
     os.close(fd)
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+    objdir = tempfile.mkdtemp(prefix="dcp_build_")
+    srcs = sources()
+    objs = [os.path.join(objdir, os.path.basename(src) + ".o") for src in srcs]
+    compiles = [[nvcc(), *ARCH, *COMPILE_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+                for src, obj in zip(srcs, objs)]
+    link = [nvcc(), *ARCH, *LINK_FLAGS, "-o", tmp, *objs]
     try:
-        res = subprocess.run(cmd, capture_output=True, text=True)
-        if res.returncode != 0:
-            raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
+        with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+            for f in [ex.submit(_run, c) for c in compiles]:
+                f.result()
+        _run(link)
         if verbose:
-            print(" ".join(cmd))
+            for c in compiles + [link]:
+                print(" ".join(c))
         os.replace(tmp, LIBRARY)
     finally:
         if os.path.exists(tmp):
             os.unlink(tmp)
+        shutil.rmtree(objdir, ignore_errors=True)
     return LIBRARY
-
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()

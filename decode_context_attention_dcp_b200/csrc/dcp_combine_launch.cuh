@@ -1,0 +1,92 @@
+// dcp_combine_launch.cuh -- choice of the combine kernel instance for a call and its
+// launch; included by the per-element-type translation units only.
+#pragma once
+
+#include "dcp_host.h"
+
+namespace dcp_host {
+
+template <class T, int G, int CPL, int NB, bool PACKED, int MIN_CTAS, bool UNIFORM, bool VARLEN, bool PACK_OUT,
+          bool PREFETCH>
+int32_t launch_combine(const dcp::CombineArgs &a, cudaStream_t stream) {
+    const char *fn = PACKED ? "dcp_unpack_combine" : PACK_OUT ? "dcp_combine_pack" : "dcp_lse_combine";
+    auto kernel = dcp::combine_kernel<T, G, CPL, NB, PACKED, MIN_CTAS, UNIFORM, VARLEN, PACK_OUT, PREFETCH>;
+    static InstanceCache ic;
+    constexpr int kUnitsPerWarp = 32 / G;
+    constexpr int kWarps = dcp::kCombineThreads / 32;
+    const size_t smem = dcp::combine_smem_bytes(kUnitsPerWarp, a.N, PACKED, PREFETCH);
+    if (!reserve_smem(kernel, ic, dcp::combine_smem_bytes(kUnitsPerWarp, DCP_MAX_SHARDS, PACKED, PREFETCH)))
+        return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
+    const int per_sm = cached_resident_ctas(kernel, ic, dcp::kCombineThreads, smem);
+    const int64_t tasks = (a.units + kUnitsPerWarp - 1) / kUnitsPerWarp;
+    const int64_t want = (tasks + kWarps - 1) / kWarps;
+    const int64_t cap = (int64_t)sm_count() * per_sm;
+    const int grid = (int)(want < cap ? want : cap);
+    kernel<<<grid, dcp::kCombineThreads, smem, stream>>>(a);
+    return launch_status(fn);
+}
+
+// Occupancy: the kernel keeps NB * CPL 16-byte loads in flight per lane, so the
+// bytes in flight per SM are set by how many warps fit.  Capping registers so
+// that 3 CTAs fit (2 for the four-slot shapes, which spill otherwise) measured
+// best on B200 for every shape.
+template <class T, int G, bool PACKED, bool UNIFORM, bool VARLEN, bool PACK_OUT, bool PREFETCH>
+int32_t launch_cpl(dcp::CombineArgs a, int cpl, cudaStream_t stream) {
+    switch (cpl) {
+        case 1: return launch_combine<T, G, 1, 8, PACKED, 3, UNIFORM, VARLEN, PACK_OUT, PREFETCH>(a, stream);
+        case 2: return launch_combine<T, G, 2, 4, PACKED, 3, UNIFORM, VARLEN, PACK_OUT, PREFETCH>(a, stream);
+        default: return launch_combine<T, G, 4, 2, PACKED, 2, UNIFORM, VARLEN, PACK_OUT, PREFETCH>(a, stream);
+    }
+}
+
+template <class T, bool PACKED, bool UNIFORM, bool VARLEN, bool PACK_OUT, bool PREFETCH>
+int32_t launch_g(dcp::CombineArgs a, int G, int cpl, cudaStream_t stream) {
+    switch (G) {
+        case 4: return launch_cpl<T, 4, PACKED, UNIFORM, VARLEN, PACK_OUT, PREFETCH>(a, cpl, stream);
+        case 8: return launch_cpl<T, 8, PACKED, UNIFORM, VARLEN, PACK_OUT, PREFETCH>(a, cpl, stream);
+        case 16: return launch_cpl<T, 16, PACKED, UNIFORM, VARLEN, PACK_OUT, PREFETCH>(a, cpl, stream);
+        default: return launch_cpl<T, 32, PACKED, UNIFORM, VARLEN, PACK_OUT, PREFETCH>(a, cpl, stream);
+    }
+}
+
+// Shape of the work per lane.  Each lane should keep about eight 16-byte loads
+// in flight: chunk slots per lane (CPL) times shards per batch (NB = 8 / CPL),
+// so fewer shards ask for more chunks per lane, i.e. fewer lanes per row (G).
+// When all shards of the packed buffer put a row at the same offset from a
+// 16-byte boundary (the shard stride is a multiple of 16 bytes) and one pass
+// covers a row, the sums are realigned once per output chunk ("uniform");
+// otherwise every shard's chunk is realigned, and that path keeps at least two
+// slots per lane.
+template <class T, bool PACKED>
+int32_t dispatch_combine(dcp::CombineArgs a, cudaStream_t stream) {
+    const int chunks = a.chunks;
+    const bool uniform = PACKED && (a.N == 1 || a.shard_stride_w % 4 == 0) && chunks <= 4 * 32;
+    int cpl_target = a.N >= 8 ? 1 : a.N >= 4 ? 2 : 4;
+    if (PACKED && !uniform && cpl_target < 2) cpl_target = 2;
+    // split layout, 8-15 shards, rows of at most 256 bytes: two chunk slots per lane (four
+    // rows per warp) measured 3-6% faster than one; packed rows lose with more slots
+    if (!PACKED && a.N >= 8 && a.N < 16 && chunks <= 16) cpl_target = 2;
+    const int per_lane = (chunks + cpl_target - 1) / cpl_target;
+    int G = 4;
+    while (G < per_lane && G < 32) G *= 2;
+    a.slots = (chunks + G - 1) / G;
+    const int cpl = a.slots >= 3 ? 4 : a.slots;  // one pass whenever slots <= 4
+    // Phase 1's reads one task ahead: measured worth it where phase 1's latency is exposed
+    // (two shards, or packed rows of 1 KiB and more), and 2-4% slower where the stream
+    // already hides it.
+    const bool prefetch = a.N <= 2 || (PACKED && chunks >= 64);
+    if constexpr (PACKED) {
+        if (uniform) {
+            if (prefetch) return launch_g<T, true, true, false, false, true>(a, G, cpl, stream);
+            return launch_g<T, true, true, false, false, false>(a, G, cpl, stream);
+        }
+        return launch_g<T, true, false, false, false, false>(a, G, cpl, stream);
+    } else {
+        if (a.varlen) return launch_g<T, false, false, true, false, true>(a, G, cpl, stream);
+        if (a.pack_b > 0) return launch_g<T, false, false, false, true, false>(a, G, cpl, stream);
+        if (prefetch) return launch_g<T, false, false, false, false, true>(a, G, cpl, stream);
+        return launch_g<T, false, false, false, false, false>(a, G, cpl, stream);
+    }
+}
+
+}  // namespace dcp_host

@@ -174,7 +174,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits that time out: counted here, read (and cleared) by the host with dcp_wait_timeouts.
-__device__ unsigned long long g_wait_timeouts = 0;
+// Internal to each translation unit: the pack kernel and dcp_wait_timeouts share one.
+static __device__ unsigned long long g_wait_timeouts = 0;
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // one second
 
