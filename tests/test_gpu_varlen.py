@@ -185,3 +185,16 @@ def test_varlen_errors():
         dcp.lse_weighted_combine_varlen(x, lse, sl, q[:2])
     with pytest.raises(ValueError):
         dcp.lse_weighted_combine_varlen(x, lse, sl.long(), q)
+
+
+@pytest.mark.parametrize("dtype,D,N", [("bf16", 2048, 4), ("fp32", 1024, 3), ("fp16", 8192, 2), ("bf16", 512, 64)])
+def test_varlen_wide_rows(o, dtype, D, N):
+    """Rows that take several passes per lane group (and the most shards): the shards without
+    KV are skipped in every pass."""
+    B, H = 23, 2
+    w = wl.CombineWorkload(f"varlen_wide_{dtype}_D{D}_N{N}", N=N, B=B, Hr=H, D=D, dtype=dtype, lse_lo=-5.0,
+                           lse_hi=15.0, p_neginf=0.05, seed=D + N)
+    outputs, lses = wl.split_inputs(w)
+    seq_lens, qsl = wl.decode_batch(wl.DecodeBatch(B=B, max_q=2, pad=3, p_short=0.6, short_max=N, max_seq=4 * N,
+                                                   seed=D + N))
+    check_varlen(o, outputs, lses, seq_lens, qsl, 1, True, w.name)
