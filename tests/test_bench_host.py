@@ -88,3 +88,33 @@ def test_max_over_ranks_gloo_world2():
     assert out[0][0] == 3.0 and out[1][0] == 3.0
     assert out[0][1] and out[1][1]
     assert out[0][2] == out[1][2] == (4, 16, 128)
+
+
+def test_kernel_digest_tracks_code_not_comments(tmp_path, monkeypatch):
+    """The digest that gates reported DRAM traffic changes with the kernel code and only with
+    it: comments and whitespace do not count, a changed token does."""
+    import shutil
+    for sub in ("decode_context_attention_dcp_b200/csrc", "include"):
+        shutil.copytree(os.path.join(ROOT, sub), tmp_path / sub)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    base = bench.kernel_digest()
+    k = tmp_path / "decode_context_attention_dcp_b200/csrc/dcp_kernels.cuh"
+    text = k.read_text()
+    k.write_text("// an added comment\n/* and a block\n   comment */\n" + text.replace("\n", "\n\n", 5))
+    assert bench.kernel_digest() == base
+    k.write_text(text.replace("kPackStages = 3", "kPackStages = 4", 1))
+    assert bench.kernel_digest() != base
+
+
+def test_traffic_is_reported_only_for_the_current_code(tmp_path, monkeypatch):
+    """load_traffic returns the committed counters while their digest matches the sources and
+    None once the code differs."""
+    import shutil
+    for sub in ("decode_context_attention_dcp_b200/csrc", "include", "profiles"):
+        shutil.copytree(os.path.join(ROOT, sub), tmp_path / sub)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    have = bench.load_traffic("dcp_pack", "sweep_N16_B16384_D512")
+    k = tmp_path / "decode_context_attention_dcp_b200/csrc/dcp_kernels.cuh"
+    k.write_text(k.read_text().replace("kPackStages = 3", "kPackStages = 4", 1))
+    assert bench.load_traffic("dcp_pack", "sweep_N16_B16384_D512") is None
+    assert have is None or have > 0
