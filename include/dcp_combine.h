@@ -44,7 +44,8 @@
  *     the calling thread; the caller owns every buffer.  The library allocates
  *     nothing.
  *   - Calls are asynchronous on `cuda_stream` (a cudaStream_t; NULL = the
- *     legacy default stream) and never synchronise.  Inputs must stay valid
+ *     legacy default stream) and never synchronise (dcp_wait_timeouts, which
+ *     reads a device counter, is the one exception).  Inputs must stay valid
  *     and outputs untouched until the stream reaches the call.
  *   - Outputs must not overlap inputs.
  *   - Sizes and strides are in ELEMENTS of the named array's type.
@@ -110,6 +111,10 @@ int32_t dcp_lse_pack_dim(int32_t dtype);
  * send_buf 16-byte aligned, out_stride_b / out_stride_h multiples of
  * 16/elemsize and >= 1 (else DCP_ERR_MISALIGNED / DCP_ERR_INVALID_ARG);
  * cp_attn_lse 4-byte aligned, lse_stride_b >= H.
+ *
+ * The kernel waits for its bulk copies with a time limit; a wait that runs out
+ * (never, while the copies work) leaves this call's send_buf incomplete and
+ * is counted by dcp_wait_timeouts.
  */
 int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_buf,
                  int64_t B, int64_t H, int64_t D, int32_t world_size, int32_t dtype,
