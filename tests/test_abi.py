@@ -231,3 +231,31 @@ def test_combine_pack_rejections(lib):
     assert _combine_pack(lib, outputs=None) == INVALID
     assert _combine_pack(lib, lses=A + 2) == MISALIGNED
     assert "dcp_combine_pack" in dcp.dcp_last_error()
+
+
+def test_error_text_is_per_thread(lib):
+    """dcp_last_error belongs to the calling thread: a failing call on one thread does not
+    change what another thread sees."""
+    import threading
+    seen = {}
+    barrier = threading.Barrier(2)
+
+    def failing():
+        assert _combine(lib, dtype=9) == DTYPE
+        barrier.wait()
+        barrier.wait()
+        seen["failing"] = dcp.dcp_last_error()
+
+    def clean():
+        assert _combine(lib, B=0) == OK
+        barrier.wait()
+        seen["clean"] = dcp.dcp_last_error()
+        barrier.wait()
+
+    ts = [threading.Thread(target=failing), threading.Thread(target=clean)]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    assert "unsupported dtype" in seen["failing"]
+    assert seen["clean"] == ""

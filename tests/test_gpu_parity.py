@@ -488,3 +488,48 @@ def test_pack_edge_shapes(o, B, H, D, ws, dtype):
     ref = o.pack(raw(out.contiguous()), raw(lse.contiguous()), ws, ORACLE_CODE[dt])
     assert np.array_equal(bits(send.tensor.cpu()), bits(ref))
     assert dcp.dcp_wait_timeouts() == 0
+
+
+def test_concurrent_host_threads(o):
+    """Four host threads, each with its own stream and inputs, pack and combine at the same
+    time (first calls included, which set up each kernel instance): every result matches the
+    oracle."""
+    import threading
+    cases = [wl.CombineWorkload(f"thr{i}", N=N, B=B, Hr=Hr, D=D, dtype=dt, lse_lo=-5.0, lse_hi=15.0, p_neginf=0.05,
+                                seed=70 + i)
+             for i, (N, B, Hr, D, dt) in enumerate([(4, 300, 8, 128, "bf16"), (8, 120, 4, 512, "fp16"),
+                                                    (2, 500, 16, 64, "fp32"), (16, 64, 2, 256, "bf16")])]
+    inputs = [wl.split_inputs(w) for w in cases]
+    results = [None] * len(cases)
+    errors = []
+    start = threading.Barrier(len(cases))
+
+    def work(i):
+        try:
+            w = cases[i]
+            outputs, lses = inputs[i]
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                d_out, d_lse = outputs.cuda(), lses.cuda()
+                start.wait()
+                y, g = dcp.lse_weighted_combine(d_out, d_lse, return_lse=True)
+                cp_out = d_out.permute(1, 0, 2, 3).reshape(w.B, w.H, w.D).contiguous()
+                cp_lse = d_lse.permute(1, 0, 2).reshape(w.B, w.H).contiguous()
+                y2, g2 = dcp.unpack_combine(dcp.pack(cp_out, cp_lse, w.N), return_lse=True)
+            s.synchronize()
+            results[i] = (y.cpu(), g.cpu(), y2.cpu(), g2.cpu())
+        except Exception as e:  # reported on the main thread
+            errors.append(e)
+
+    ts = [threading.Thread(target=work, args=(i,)) for i in range(len(cases))]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    assert not errors, errors
+    for w, (outputs, lses), (y, g, y2, g2) in zip(cases, inputs, results):
+        ry, rg = o.lse_combine(raw(outputs), ORACLE_CODE[outputs.dtype], raw(lses), return_lse=True)
+        assert_out_close(y, ry, f"{w.name} combine")
+        assert_lse_close(g, rg, f"{w.name} combine lse")
+        assert_out_close(y2, ry, f"{w.name} pack + unpack_combine")
+        assert_lse_close(g2, rg, f"{w.name} pack + unpack_combine lse")
