@@ -14,8 +14,10 @@ draws taken in this order):
      p_neginf <= u < p_neginf + p_nan gives the quiet NaN 0x7FC00000;
   4. structured holes: for ``empty_every = k``, every token b with b % k == 0
      has -inf at every shard (an empty KV context).
-Large tensors are drawn in token slices, in token order, so memory stays bounded
-and the bits are the same whatever the slice size.
+Large tensors are drawn in token slices, in token order, so memory stays bounded.
+The slice size is a fixed function of the workload's shape (about 2^24 elements per
+slice), so a workload's bits are reproducible; a different slicing would draw different
+bits.
 """
 from __future__ import annotations
 

@@ -118,3 +118,20 @@ def test_traffic_is_reported_only_for_the_current_code(tmp_path, monkeypatch):
     k.write_text(k.read_text().replace("kPackStages = 3", "kPackStages = 4", 1))
     assert bench.load_traffic("dcp_pack", "sweep_N16_B16384_D512") is None
     assert have is None or have > 0
+
+
+def test_workload_inputs_are_reproducible():
+    """The same workload draws the same bits every time (the seeded generators are the only
+    source of the inputs both sides see)."""
+    from decode_context_attention_dcp_b200 import workloads as wl
+    w = wl.CombineWorkload("repro", N=3, B=40, Hr=4, D=64, p_neginf=0.1, p_nan=0.05, empty_every=7, seed=11)
+    a, b = wl.split_inputs(w), wl.split_inputs(w)
+    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
+    assert torch.equal(a[1].view(torch.int32), b[1].view(torch.int32))
+    c, d = wl.pack_inputs(w), wl.pack_inputs(w)
+    assert torch.equal(c[0].view(torch.int16), d[0].view(torch.int16))
+    assert torch.equal(c[1].view(torch.int32), d[1].view(torch.int32))
+    s1, q1 = wl.decode_batch(wl.DecodeBatch(B=50, max_q=3, pad=4, seed=3))
+    s2, q2 = wl.decode_batch(wl.DecodeBatch(B=50, max_q=3, pad=4, seed=3))
+    assert torch.equal(s1, s2) and torch.equal(q1, q2) and int(q1[-1]) == 46 and int(q1[0]) == 0
+    assert bool((q1[1:] > q1[:-1]).all()) and bool(((q1[1:] - q1[:-1]) <= 3).all())
