@@ -375,3 +375,27 @@ def pin_varlen_reduces_to_combine(o: orc.Oracle) -> None:
 
 
 ALL_PINS.append(pin_varlen_reduces_to_combine)
+
+
+def pin_varlen_golden(o: orc.Oracle) -> None:
+    """Hand-derived worked examples of the variable-length reading (tests/golden)."""
+    with open(os.path.join(GOLDEN, "varlen_worked_examples.json")) as fh:
+        cases = json.load(fh)["cases"]
+    for c in cases:
+        outs = np.asarray([[[_f(x) for x in row] for row in shard] for shard in c["outputs"]], dtype=np.float32)
+        N, T, D = outs.shape
+        raw = bf16_bits(outs.reshape(-1)).reshape(N, T, 1, D)
+        lses = np.asarray(c["lses"], dtype=np.float32).reshape(N, T, 1)
+        y, g = o.lse_combine_varlen(raw, orc.BF16, lses, c["seq_lens"], c["query_start_loc"], c["interleave"],
+                                    return_lse=True, is_lse_base_on_e=c["base_e"])
+        np.testing.assert_allclose(y.reshape(T, D), np.asarray(c["result"], dtype=np.float64), rtol=0, atol=1e-12,
+                                   err_msg=c["name"])
+        for t, want in enumerate(c["global_lse"]):
+            want = _f(want)
+            if math.isinf(want):
+                assert g[t, 0] == want, (c["name"], t, g[t, 0])
+            else:
+                assert abs(g[t, 0] - want) <= 1e-12, (c["name"], t, g[t, 0], want)
+
+
+ALL_PINS.append(pin_varlen_golden)
