@@ -64,7 +64,7 @@ def assert_lse_close(gpu: torch.Tensor, ref: np.ndarray, what: str = "") -> None
     assert np.array_equal(np.isinf(got), inf_ref), f"{what}: infinite global LSEs differ"
     assert np.array_equal(got[inf_ref], ref[inf_ref]), f"{what}: -inf must stay -inf"
     assert not np.isnan(got).any(), f"{what}: NaN global LSE"
-    err = np.abs(got - ref)[~inf_ref]
+    err = np.abs(got[~inf_ref] - ref[~inf_ref])
     assert err.size == 0 or err.max() <= LSE_TOL, f"{what}: global LSE err {err.max():.3g} > {LSE_TOL}"
 
 
