@@ -359,7 +359,8 @@ int64_t oracle_local_seq_len(int64_t seq_len, int64_t cp_size, int64_t rank, int
  *     request have no context at all;
  *   - shard n holds oracle_local_seq_len(seq_lens[r], N, n, interleave) KV
  *     positions of request r ([ASC] _get_dcp_local_seq_lens); a shard that
- *     holds none is empty: its LSE counts as -inf and its output row is not
+ *     holds none (a local length <= 0, which a negative seq_lens entry gives) is
+ *     empty: its LSE counts as -inf and its output row is not
  *     read (it may never have been written);
  *   - everything else is oracle_lse_combine.
  * Same layouts as oracle_lse_combine (split layout, shard strides).
@@ -380,7 +381,7 @@ int oracle_lse_combine_varlen(const void *outputs, int out_dtype, const void *ls
         for (int r = 0; r < num_reqs; ++r)
             if (query_start_loc[r] <= b && b < query_start_loc[r + 1]) req = r;
         for (int n = 0; n < N; ++n)
-            empty[n] = req < 0 || oracle_local_seq_len(seq_lens[req], N, n, interleave) == 0;
+            empty[n] = req < 0 || oracle_local_seq_len(seq_lens[req], N, n, interleave) <= 0;
         for (int64_t h = 0; h < H; ++h)
             combine_row(outputs, out_dtype, lses, lse_dtype, result, global_lse, N, b, h, B, H, D,
                         out_stride_n, lse_stride_n, is_lse_base_on_e, return_lse, empty, l, w);
