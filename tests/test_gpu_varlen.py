@@ -111,11 +111,12 @@ def test_varlen_without_requests(o):
 
 
 def test_varlen_zero_length_requests(o):
-    """Requests whose KV length is 0 combine no shard; their neighbours are unaffected."""
+    """Requests whose KV length is 0 (or negative) combine no shard; their neighbours are
+    unaffected."""
     N, B, H, D = 4, 6, 2, 64
     w = wl.CombineWorkload("varlen_zero", N=N, B=B, Hr=H, D=D, seed=43)
     outputs, lses = wl.split_inputs(w)
-    seq_lens = torch.tensor([0, 3, 0, 100, 1], dtype=torch.int32)
+    seq_lens = torch.tensor([0, 3, -100, 100, 1], dtype=torch.int32)
     qsl = torch.tensor([0, 1, 2, 4, 5, 6], dtype=torch.int32)
     y, g, _ = check_varlen(o, outputs, lses, seq_lens, qsl, 1, what="zero-length")
     assert bool((y[0] == 0).all()) and bool((y[2:4] == 0).all())
