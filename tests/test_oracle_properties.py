@@ -101,3 +101,20 @@ def test_repeated_shard_is_a_larger_lse(c, k):
     yb, gb = o().lse_combine(raw, code, bumped, return_lse=True, is_lse_base_on_e=c["base_e"])
     _close(y, yb, 1e-12)
     _close(g, gb, 1e-12)
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.integers(0, 20000), st.integers(1, 64), st.sampled_from([1, 2, 3, 4, 16, 64, 128]))
+def test_shards_holding_kv_are_a_prefix(seq, N, interleave):
+    """Under interleaved sharding (vllm-ascend sfa_cp.py _get_dcp_local_seq_lens) shard n holds
+    positions of a request of length seq exactly when n * interleave < seq, so the shards
+    holding KV are shards [0, k) with k = min(N, ceil(seq / interleave)) -- the criterion the
+    variable-length kernels evaluate instead of the local length -- and the local lengths add
+    up to seq."""
+    lens = [o().local_seq_len(seq, N, n, interleave) for n in range(N)]
+    assert sum(lens) == seq
+    assert all(ln >= 0 for ln in lens)
+    for n, ln in enumerate(lens):
+        assert (ln > 0) == (n * interleave < seq), (seq, N, interleave, n, ln)
+    k = min(N, -(-seq // interleave))
+    assert [ln > 0 for ln in lens] == [n < k for n in range(N)]
