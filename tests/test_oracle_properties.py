@@ -5,7 +5,8 @@ softmax-weighted mean over the shard axis.  Whatever the shapes, values, base an
 it must be invariant under a permutation of the shards, invariant (output) and equivariant
 (global LSE) under one shift of every LSE, agree with the softmax statement of the same merge
 in vllm-ascend sfa_cp.py _merge_dcp_outputs_with_torch, and treat a shard repeated k times
-like one shard whose LSE is larger by log k.  Hypothesis draws the cases.
+like one shard whose LSE is larger by log k.  The interleaved sharding of the variable-length
+reading puts KV on a prefix of the shards.  Hypothesis draws the cases.
 """
 from __future__ import annotations
 
