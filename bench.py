@@ -14,8 +14,16 @@ stream), max over ranks; also (token*head)/s and the fraction of the measured HB
 With N > 1 (torchrun, one process per GPU) every rank combines its own batch: weak scaling,
 no data-path collective.  Rank 0 prints one JSON line.
 
+The line also carries: per-kernel times and shares; "roofline" (the dominant kernel's
+achieved GB/s against the measured copy peak, with ncu DRAM traffic when the committed
+summary was taken on the current kernel code); "e2e" (the same step through the public API
+with pinned host inputs copied in and the result copied out every step); "cpu_baseline"
+(the oracle on a bounded token slice, one host core, N = 1 only); "gpu_launches"; and the SM
+clocks sampled during the timed region.
+
 --impl reference times the fp64 CPU oracle on the host cores on a bounded sample of the same
-workload (rank 0 only), for the same metric.
+workload (rank 0 only), for the same metric.  --sweep times every entry point on every
+workload (median of launches with L2 flushed before each) and prints a markdown table.
 """
 from __future__ import annotations
 
