@@ -14,6 +14,10 @@
  *   [ASC]   vllm-ascend, vllm_ascend/attention/context_parallel/sfa_cp.py:
  *           _merge_dcp_outputs_with_torch (the same merge written as a softmax
  *           over the shard axis) and _get_dcp_local_seq_lens (KV sharding).
+ *   [DIRECT] vLLM API docs, module vllm.v1.attention.ops.dcp:
+ *           DirectDCPA2AWorkspace.lse_reduce, which also takes seq_lens and
+ *           query_start_loc; oracle_lse_combine_varlen implements a stated
+ *           reading of them (parity of that reading is unpinned).
  *
  * Everything is written as the definition, step by step, in double precision.
  * Loops run in the natural index order; there is no blocking, fusion or
