@@ -18,11 +18,11 @@ The line also carries: per-kernel times and shares; "roofline" (the dominant ker
 achieved GB/s against the measured copy peak, with ncu DRAM traffic when the committed
 summary was taken on the current kernel code); "e2e" (the same step through the public API
 with pinned host inputs copied in and the result copied out every step); "cpu_baseline"
-(the oracle on a bounded token slice, one host core, N = 1 only); "gpu_launches"; and the SM
+(the oracle on a bounded token sample, on all host cores and on one, N = 1 only); "gpu_launches"; and the SM
 clocks sampled during the timed region.
 
---impl reference times the fp64 CPU oracle on the host cores on a bounded sample of the same
-workload (rank 0 only), for the same metric.  --sweep times every entry point on every
+--impl reference times the fp64 CPU oracle on all host cores (token slices, one thread each) on
+the same bounded sample of the workload as the CPU baseline (rank 0 only), for the same metric.  --sweep times every entry point on every
 workload (median of launches with L2 flushed before each) and prints a markdown table.
 """
 from __future__ import annotations
@@ -194,38 +194,97 @@ class ClockSampler:
 
 
 # ---- the CPU oracle (reference arm and CPU baseline) -----------------------------------------
-def oracle_step_sample(w, tokens: int):
-    """One oracle step (pack + unpack+combine, plain fp64 C) on the first ``tokens`` tokens of the
-    workload's rank-0 inputs.  Returns (seconds, algorithmic bytes)."""
-    import numpy as np
-    import torch
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+
+
+def cpu_sample_tokens(w) -> int:
+    """Tokens of the oracle's sample: one eighth of the batch, at most 2048 (both the CPU baseline
+    and the reference arm use this sample)."""
+    return max(1, min(2048, w.B // 8 or w.B))
+
+
+_SAMPLES: dict = {}
+
+
+def oracle_sample(w, tokens: int):
+    """The sample's inputs as the oracle reads them: a ``tokens``-token batch drawn with the
+    workload's recipe and seed (cp_attn_out [tokens, H, D] raw elements, cp_attn_lse fp32)."""
+    key = (w, tokens)
+    if key not in _SAMPLES:
+        import numpy as np
+        import torch
+
+        from decode_context_attention_dcp_b200 import workloads as wl
+
+        cp_out, cp_lse = wl.pack_inputs(w.with_(B=tokens))
+        ro = cp_out.view(torch.int16).numpy().view(np.uint16) if cp_out.element_size() == 2 else cp_out.numpy()
+        _SAMPLES.clear()
+        _SAMPLES[key] = (ro, cp_lse.numpy())
+    return _SAMPLES[key]
+
+
+def oracle_step_sample(w, tokens: int, threads: int = 1):
+    """One oracle step (pack, then unpack+combine, plain fp64 C) over the sample.  With
+    ``threads`` > 1 the tokens are split into that many slices and each host thread runs both
+    steps of the unchanged oracle on its own slice (ctypes releases the GIL).  Returns
+    (seconds, algorithmic bytes)."""
+    import concurrent.futures
 
     import oracle
-    from decode_context_attention_dcp_b200 import workloads as wl
 
-    ws = w.with_(B=tokens)
-    cp_out, cp_lse = wl.pack_inputs(ws)
+    ro, rl = oracle_sample(w, tokens)
     o = oracle.load()
-    code = {torch.bfloat16: oracle.BF16, torch.float16: oracle.FP16, torch.float32: oracle.FP32}[cp_out.dtype]
-    ro = cp_out.view(torch.int16).numpy().view(np.uint16) if cp_out.element_size() == 2 else cp_out.numpy()
+    code = {"bf16": oracle.BF16, "fp16": oracle.FP16, "fp32": oracle.FP32}[w.dtype]
+
+    def run(t0: int, t1: int) -> None:
+        send = o.pack(ro[t0:t1], rl[t0:t1], w.N, code)
+        o.unpack_combine(send, code, w.D, return_lse=w.return_lse, is_lse_base_on_e=w.is_lse_base_on_e)
+
+    threads = max(1, min(threads, tokens))
+    step = (tokens + threads - 1) // threads
+    bounds = [(t, min(tokens, t + step)) for t in range(0, tokens, step)]
     t0 = time.perf_counter()
-    send = o.pack(ro, cp_lse.numpy(), ws.N, code)
-    o.unpack_combine(send, code, ws.D, return_lse=ws.return_lse, is_lse_base_on_e=ws.is_lse_base_on_e)
+    if len(bounds) == 1:
+        run(*bounds[0])
+    else:
+        with concurrent.futures.ThreadPoolExecutor(max_workers=len(bounds)) as ex:
+            for f in [ex.submit(run, a, b) for a, b in bounds]:
+                f.result()
     dt = time.perf_counter() - t0
+    ws = w.with_(B=tokens)
     return dt, ws.pack_bytes() + ws.combine_bytes()
 
 
-def cpu_baseline(w, budget_s: float = 12.0) -> dict:
-    tokens = max(1, w.B // 8)
+def time_oracle(w, tokens: int, threads: int, budget_s: float, max_reps: int) -> tuple[float, int, float]:
+    """(GB/s, repetitions, seconds) of oracle steps over the sample until the budget is spent."""
     total_t, total_b, reps = 0.0, 0, 0
-    while total_t < budget_s and reps < 8:
-        dt, nb = oracle_step_sample(w, tokens)
+    while reps < 1 or (total_t < budget_s and reps < max_reps):
+        dt, nb = oracle_step_sample(w, tokens, threads)
         total_t += dt
         total_b += nb
         reps += 1
-    return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{reps} x (pack + unpack_combine) of the first {tokens} of {w.B} tokens, "
-                      f"single-threaded fp64 C, {total_t:.1f} s"}
+    return total_b / total_t / 1e9, reps, total_t
+
+
+def sample_text(w, tokens: int) -> str:
+    return (f"pack + unpack_combine of a {tokens}-token batch drawn with the workload's recipe "
+            f"({tokens} of {w.B} tokens, all {w.N} shards, Hr={w.Hr}, D={w.D}); plain fp64 C")
+
+
+def cpu_baseline(w, budget_s: float = 12.0) -> dict:
+    """The oracle on the host's cores (all of them, token slices), and on one core, over the
+    same sample."""
+    tokens = cpu_sample_tokens(w)
+    cores = host_cores()
+    oracle_step_sample(w, tokens, cores)  # inputs drawn, pages touched
+    v_all, r_all, t_all = time_oracle(w, tokens, cores, budget_s / 2, 32)
+    v_one, r_one, t_one = time_oracle(w, tokens, 1, budget_s / 2, 8)
+    return {"value": v_all, "unit": "GB/s", "cores": cores, "kind": "oracle", "host_cores": os.cpu_count(),
+            "sample": f"{sample_text(w, tokens)}; {r_all} steps on {cores} threads ({t_all:.1f} s)",
+            "single_thread": {"value": v_one, "unit": "GB/s", "cores": 1,
+                              "sample": f"the same sample, {r_one} steps on one thread ({t_one:.1f} s)"}}
 
 
 def run_reference(args) -> int:
@@ -235,22 +294,27 @@ def run_reference(args) -> int:
     from decode_context_attention_dcp_b200 import workloads as wl
 
     w = wl.by_name(args.workload)
-    tokens = max(1, min(w.B, 256))
+    tokens = cpu_sample_tokens(w)
+    cores = host_cores()
     for _ in range(args.warmup):
-        oracle_step_sample(w, tokens)
+        oracle_step_sample(w, tokens, cores)
     secs, nbytes = 0.0, 0
     for _ in range(args.steps):
-        dt, nb = oracle_step_sample(w, tokens)
+        dt, nb = oracle_step_sample(w, tokens, cores)
         secs += dt
         nbytes += nb
     gbs = nbytes / secs / 1e9
-    sample = f"each step: pack + unpack_combine of the first {tokens} of {w.B} tokens, single-threaded fp64 C"
+    v_one, r_one, t_one = time_oracle(w, tokens, 1, 4.0, 4)
+    sample = f"each step: {sample_text(w, tokens)}, token slices on {cores} threads"
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w),
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample,
+                         "host_cores": os.cpu_count(),
+                         "single_thread": {"value": v_one, "unit": "GB/s", "cores": 1,
+                                           "sample": f"the same sample, {r_one} steps on one thread ({t_one:.1f} s)"}},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }

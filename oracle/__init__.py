@@ -17,7 +17,9 @@ Sources, by page and section:
 """
 from __future__ import annotations
 
+import concurrent.futures
 import ctypes
+import hashlib
 import os
 import subprocess
 import tempfile
@@ -36,16 +38,26 @@ _c_int = ctypes.c_int
 _c_ptr = ctypes.c_void_p
 
 
+_GCC_FLAGS = ["-O2", "-fno-fast-math", "-std=c11", "-fPIC", "-shared"]
+
+
+def _digest(source: str) -> str:
+    h = hashlib.sha256(" ".join(_GCC_FLAGS).encode() + b"\0")
+    with open(source, "rb") as fh:
+        h.update(fh.read())
+    return h.hexdigest()
+
+
 def compile_oracle(source: str = SOURCE, output: str = LIBRARY) -> str:
-    """Compile the C oracle into a shared library (atomically replaces ``output``)."""
+    """Compile the C oracle into a shared library (atomically replaces ``output``; the source's
+    digest is kept beside it)."""
     fd, tmp = tempfile.mkstemp(suffix=".so", dir=os.path.dirname(output))
     os.close(fd)
     try:
-        subprocess.run(
-            ["gcc", "-O2", "-fno-fast-math", "-std=c11", "-fPIC", "-shared", "-o", tmp, source, "-lm"],
-            check=True,
-        )
+        subprocess.run(["gcc", *_GCC_FLAGS, "-o", tmp, source, "-lm"], check=True)
         os.replace(tmp, output)
+        with open(output + ".sha256", "w") as fh:
+            fh.write(_digest(source) + "\n")
     finally:
         if os.path.exists(tmp):
             os.unlink(tmp)
@@ -53,7 +65,11 @@ def compile_oracle(source: str = SOURCE, output: str = LIBRARY) -> str:
 
 
 def _stale(lib: str, src: str) -> bool:
-    return not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src)
+    """True unless ``lib`` was built from exactly the current source and flags."""
+    if not os.path.exists(lib) or not os.path.exists(lib + ".sha256"):
+        return True
+    with open(lib + ".sha256") as fh:
+        return fh.read().strip() != _digest(src)
 
 
 class Oracle:
@@ -160,27 +176,6 @@ class Oracle:
         self._check(rc, "lse_combine")
         return (result, glse) if return_lse else result
 
-    def lse_combine_rows(self, outputs: np.ndarray, out_dtype: int, lses: np.ndarray, rows,
-                         return_lse: bool = False, is_lse_base_on_e: bool = True):
-        """The combine of selected (b, h) rows only, read in place from full-size arrays.
-
-        outputs [N, B, H, D] / lses [N, B, H] must be C-contiguous; ``rows`` is a list of (b, h).
-        Returns ([len(rows), D] float64, [len(rows)] float64)."""
-        assert outputs.flags.c_contiguous and lses.flags.c_contiguous
-        N, B, H, D = outputs.shape
-        lse_dtype = F64 if lses.dtype == np.float64 else FP32
-        es, ls = outputs.dtype.itemsize, lses.dtype.itemsize
-        res = np.zeros((len(rows), D), dtype=np.float64)
-        gl = np.zeros(len(rows), dtype=np.float64)
-        for i, (b, h) in enumerate(rows):
-            unit = b * H + h
-            rc = self.lib.oracle_lse_combine(self._ptr(outputs) + unit * D * es, out_dtype,
-                                             self._ptr(lses) + unit * ls, lse_dtype,
-                                             self._ptr(res) + i * D * 8, self._ptr(gl) + i * 8,
-                                             N, 1, 1, D, B * H * D, B * H, int(is_lse_base_on_e), int(return_lse))
-            self._check(rc, "lse_combine")
-        return res, gl
-
     def unpack_combine(self, recv: np.ndarray, dtype: int, D: int, return_lse: bool = False,
                        is_lse_base_on_e: bool = True):
         recv = np.ascontiguousarray(recv)
@@ -192,21 +187,96 @@ class Oracle:
         self._check(rc, "unpack_combine")
         return (result, glse) if return_lse else result
 
-    def unpack_combine_rows(self, recv: np.ndarray, dtype: int, D: int, rows, return_lse: bool = False,
-                            is_lse_base_on_e: bool = True):
-        """unpack+combine of selected (b, h) rows, read in place from a C-contiguous [N, B, Hr, W] buffer."""
+    # ---- token slices on several host threads ------------------------------------------
+    # Every (token, head) row of the combine is independent, so a token range can be split
+    # over threads: each thread runs the unchanged C function on its own slice, addressed in
+    # place through the full arrays' shard strides.  ctypes releases the GIL during the call.
+    @staticmethod
+    def _split_run(fn, b0: int, b1: int, threads: int) -> None:
+        threads = max(1, min(threads, b1 - b0))
+        if threads == 1:
+            fn(b0, b1)
+            return
+        step = (b1 - b0 + threads - 1) // threads
+        bounds = [(s, min(b1, s + step)) for s in range(b0, b1, step)]
+        with concurrent.futures.ThreadPoolExecutor(max_workers=len(bounds)) as ex:
+            for f in [ex.submit(fn, s, e) for s, e in bounds]:
+                f.result()
+
+    def lse_combine_tokens(self, outputs: np.ndarray, out_dtype: int, lses: np.ndarray, b0: int, b1: int,
+                           return_lse: bool = False, is_lse_base_on_e: bool = True, threads: int = 1):
+        """``lse_combine`` of tokens [b0, b1) only, read in place from C-contiguous full-size
+        outputs [N, B, H, D] / lses [N, B, H]; ``threads`` host threads share the tokens.
+        Returns [b1 - b0, H, D] float64 (+ [b1 - b0, H] float64)."""
+        assert outputs.flags.c_contiguous and lses.flags.c_contiguous
+        N, B, H, D = outputs.shape
+        assert lses.shape == (N, B, H) and 0 <= b0 <= b1 <= B
+        lse_dtype = F64 if lses.dtype == np.float64 else FP32
+        es, ls = outputs.dtype.itemsize, lses.dtype.itemsize
+        result = np.zeros((b1 - b0, H, D), dtype=np.float64)
+        glse = np.zeros((b1 - b0, H), dtype=np.float64)
+
+        def run(s: int, e: int) -> None:
+            rc = self.lib.oracle_lse_combine(self._ptr(outputs) + s * H * D * es, out_dtype,
+                                             self._ptr(lses) + s * H * ls, lse_dtype,
+                                             self._ptr(result) + (s - b0) * H * D * 8,
+                                             self._ptr(glse) + (s - b0) * H * 8, N, e - s, H, D, B * H * D, B * H,
+                                             int(is_lse_base_on_e), int(return_lse))
+            self._check(rc, "lse_combine")
+
+        self._split_run(run, b0, b1, threads)
+        return (result, glse) if return_lse else result
+
+    def unpack_combine_tokens(self, recv: np.ndarray, dtype: int, D: int, b0: int, b1: int,
+                              return_lse: bool = False, is_lse_base_on_e: bool = True, threads: int = 1):
+        """``unpack_combine`` of tokens [b0, b1) only, read in place from a C-contiguous
+        [N, B, Hr, W] buffer; ``threads`` host threads share the tokens."""
         assert recv.flags.c_contiguous
         N, B, Hr, W = recv.shape
+        assert 0 <= b0 <= b1 <= B
         es = recv.dtype.itemsize
-        res = np.zeros((len(rows), D), dtype=np.float64)
-        gl = np.zeros(len(rows), dtype=np.float64)
-        for i, (b, h) in enumerate(rows):
-            unit = b * Hr + h
-            rc = self.lib.oracle_unpack_combine(self._ptr(recv) + unit * W * es, dtype, self._ptr(res) + i * D * 8,
-                                                self._ptr(gl) + i * 8, N, 1, 1, D, B * Hr * W,
+        result = np.zeros((b1 - b0, Hr, D), dtype=np.float64)
+        glse = np.zeros((b1 - b0, Hr), dtype=np.float64)
+
+        def run(s: int, e: int) -> None:
+            rc = self.lib.oracle_unpack_combine(self._ptr(recv) + s * Hr * W * es, dtype,
+                                                self._ptr(result) + (s - b0) * Hr * D * 8,
+                                                self._ptr(glse) + (s - b0) * Hr * 8, N, e - s, Hr, D, B * Hr * W,
                                                 int(is_lse_base_on_e), int(return_lse))
             self._check(rc, "unpack_combine")
-        return res, gl
+
+        self._split_run(run, b0, b1, threads)
+        return (result, glse) if return_lse else result
+
+    def lse_combine_varlen_tokens(self, outputs: np.ndarray, out_dtype: int, lses: np.ndarray, seq_lens,
+                                  query_start_loc, b0: int, b1: int, interleave: int = 1, return_lse: bool = False,
+                                  is_lse_base_on_e: bool = True, threads: int = 1):
+        """``lse_combine_varlen`` of tokens [b0, b1) only, read in place from C-contiguous
+        full-size outputs [N, B, H, D] / lses [N, B, H].  A slice starting at token s sees
+        query_start_loc - s (the same requests, indexed from the slice's first token)."""
+        assert outputs.flags.c_contiguous and lses.flags.c_contiguous
+        N, B, H, D = outputs.shape
+        assert lses.shape == (N, B, H) and 0 <= b0 <= b1 <= B
+        sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+        qsl = np.asarray(query_start_loc, dtype=np.int64)
+        assert qsl.shape[0] == sl.shape[0] + 1
+        lse_dtype = F64 if lses.dtype == np.float64 else FP32
+        es, ls = outputs.dtype.itemsize, lses.dtype.itemsize
+        result = np.zeros((b1 - b0, H, D), dtype=np.float64)
+        glse = np.zeros((b1 - b0, H), dtype=np.float64)
+
+        def run(s: int, e: int) -> None:
+            q = np.ascontiguousarray(qsl - s, dtype=np.int32)
+            rc = self.lib.oracle_lse_combine_varlen(self._ptr(outputs) + s * H * D * es, out_dtype,
+                                                    self._ptr(lses) + s * H * ls, lse_dtype,
+                                                    self._ptr(result) + (s - b0) * H * D * 8,
+                                                    self._ptr(glse) + (s - b0) * H * 8, N, e - s, H, D, B * H * D,
+                                                    B * H, self._ptr(sl) if len(sl) else None, self._ptr(q), len(sl),
+                                                    int(interleave), int(is_lse_base_on_e), int(return_lse))
+            self._check(rc, "lse_combine_varlen")
+
+        self._split_run(run, b0, b1, threads)
+        return (result, glse) if return_lse else result
 
     def softmax_merge(self, outputs: np.ndarray, out_dtype: int, lses: np.ndarray) -> np.ndarray:
         outputs = np.ascontiguousarray(outputs)

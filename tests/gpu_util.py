@@ -2,6 +2,8 @@
 construction for tests, tolerance checks, and guarded output buffers."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -13,6 +15,8 @@ import oracle as orc
 OUT_TOL = {torch.bfloat16: 1e-2, torch.float16: 1e-2, torch.float32: 2e-5}
 LSE_TOL = 1e-4
 ORACLE_CODE = {torch.bfloat16: orc.BF16, torch.float16: orc.FP16, torch.float32: orc.FP32}
+# Host threads the oracle may use on full-size inputs (token slices, see oracle.Oracle.*_tokens).
+HOST_THREADS = max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1))
 
 
 def raw(t: torch.Tensor) -> np.ndarray:
@@ -87,11 +91,16 @@ class Guarded:
         assert bool((tail == 0xA5).all()), "write past the end of the output"
 
 
-def sample_rows(B: int, H: int, count: int, seed: int, specials=()) -> list[tuple[int, int]]:
-    """``count`` (b, h) pairs spread over the batch (first and last rows included), plus ``specials``."""
-    rng = np.random.default_rng(seed)
-    rows = {(0, 0), (B - 1, H - 1), (B // 2, H // 2)}
-    while len(rows) < count:
-        rows.add((int(rng.integers(0, B)), int(rng.integers(0, H))))
-    rows.update(specials)
-    return sorted(rows)
+def compare_token_blocks(B: int, per_token_elems: int, ref_fn, outs, lses=(), what: str = "") -> None:
+    """Element-by-element comparison of full-size device results with the oracle, one block of
+    tokens at a time so host memory stays bounded.  ``ref_fn(b0, b1)`` returns the oracle's
+    (result, global LSE) of tokens [b0, b1); ``outs`` and ``lses`` list (device tensor, label)
+    pairs of [B, ...] results and global LSEs to check against them."""
+    block = max(1, (1 << 24) // max(1, per_token_elems))
+    for b0 in range(0, B, block):
+        b1 = min(B, b0 + block)
+        ry, rg = ref_fn(b0, b1)
+        for t, label in outs:
+            assert_out_close(t[b0:b1], ry, f"{what} {label} tokens [{b0}, {b1})")
+        for t, label in lses:
+            assert_lse_close(t[b0:b1], rg, f"{what} {label} tokens [{b0}, {b1})")

@@ -40,9 +40,33 @@ def test_reference_arm_prints_one_line():
     assert line["metric"] == bench.METRIC and line["unit"] == "GB/s" and line["value"] > 0
     assert line["higher_is_better"] is True
     assert line["config"]["workload"] == "sweep_N2_B512_D128"
-    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
-    assert line["cpu_baseline"]["value"] == line["value"]
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == bench.host_cores() and cb["value"] == line["value"]
+    assert cb["single_thread"]["cores"] == 1 and cb["single_thread"]["value"] > 0
+    assert f"{bench.cpu_sample_tokens(bench_workload('sweep_N2_B512_D128'))}-token" in cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def bench_workload(name):
+    from decode_context_attention_dcp_b200 import workloads as wl
+    return wl.by_name(name)
+
+
+def test_cpu_baseline_all_cores_and_one():
+    """The CPU baseline times the same sample on all host cores and on one, and states both."""
+    w = bench_workload("sweep_N2_B512_D128")
+    cb = bench.cpu_baseline(w, budget_s=1.0)
+    assert cb["kind"] == "oracle" and cb["cores"] == bench.host_cores() and cb["value"] > 0
+    assert cb["single_thread"]["cores"] == 1 and cb["single_thread"]["value"] > 0
+    assert cb["host_cores"] == os.cpu_count()
+    assert f"{bench.cpu_sample_tokens(w)}-token" in cb["sample"]
+
+
+def test_oracle_step_on_threads_moves_the_same_bytes():
+    w = bench_workload("tiny")
+    t1, b1 = bench.oracle_step_sample(w, 4, 1)
+    t2, b2 = bench.oracle_step_sample(w, 4, 3)
+    assert b1 == b2 == w.pack_bytes() + w.combine_bytes()
 
 
 def test_reference_arm_other_ranks_exit_silently():

@@ -15,7 +15,8 @@ import torch
 import decode_context_attention_dcp_b200 as dcp
 import oracle as orc
 from decode_context_attention_dcp_b200 import workloads as wl
-from gpu_util import ORACLE_CODE, Guarded, assert_lse_close, assert_out_close, bits, raw, sample_rows
+from gpu_util import (HOST_THREADS, ORACLE_CODE, Guarded, assert_lse_close, assert_out_close, bits,
+                      compare_token_blocks, raw)
 
 pytestmark = pytest.mark.gpu
 
@@ -91,23 +92,24 @@ def test_combine_pack_capacity_strided_splits(o):
     assert torch.equal(send.view(torch.int16), two_step(d_out, d_lse, ws, True).view(torch.int16))
 
 
-def test_combine_pack_large_sampled(o):
+def test_combine_pack_large_elementwise(o):
     """A flash-decoding-sized producer (S=4 splits, B=2048 tokens, H=256 heads, D=512, bf16,
-    2.1 GB of partials) into the 16-rank send buffer; sampled rows against the oracle, the
-    whole buffer against the two-step path."""
+    2.1 GB of partials) into the 16-rank send buffer: every merged row and LSE against the
+    oracle (token slices on all host cores), the whole buffer against the two-step path."""
     S, B, H, D, ws = 4, 2048, 256, 512, 16
     w = wl.CombineWorkload("cp_large", N=S, B=B, Hr=H, D=D, lse_lo=-5.0, lse_hi=25.0, p_neginf=0.02, seed=62)
     outputs, lses = wl.split_inputs(w)
     d_out, d_lse = outputs.cuda(), lses.cuda()
     send = dcp.combine_pack(d_out, d_lse, ws)
     torch.cuda.synchronize()
-    rows = sample_rows(B, H, 64, 62)
-    ref, ref_l = o.lse_combine_rows(raw(outputs), orc.BF16, raw(lses), rows, return_lse=True)
     data, lse = split_packed(send, H)
-    bi = torch.tensor([r[0] for r in rows])
-    hi = torch.tensor([r[1] for r in rows])
-    assert_out_close(data.cpu()[bi, hi], ref, "large combine_pack (sampled)")
-    assert_lse_close(lse.cpu()[bi, hi], ref_l, "large combine_pack lse (sampled)")
+    ro, rl = raw(outputs), raw(lses)
+
+    def ref(b0, b1):
+        return o.lse_combine_tokens(ro, orc.BF16, rl, b0, b1, return_lse=True, threads=HOST_THREADS)
+
+    compare_token_blocks(B, H * D, ref, [(data, "dcp_combine_pack rows")], [(lse, "dcp_combine_pack lse")],
+                         "large combine_pack")
     assert torch.equal(send.view(torch.int16), two_step(d_out, d_lse, ws, True).view(torch.int16))
 
 

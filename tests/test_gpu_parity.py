@@ -1,7 +1,7 @@
 """Parity of the CUDA path (through the C ABI) with the fp64 oracle, on the seeded DCP workloads.
 
-Element by element wherever the oracle finishes in seconds; at the largest sizes on sampled
-(token, head) rows plus properties that hold everywhere.  Pack is compared bit for bit.
+Element by element everywhere, the full-size sweep points included (the oracle runs over token
+slices on all host cores there).  Pack is compared bit for bit.
 """
 from __future__ import annotations
 
@@ -15,8 +15,8 @@ import decode_context_attention_dcp_b200 as dcp
 import oracle as orc
 import oracle_pins
 from decode_context_attention_dcp_b200 import workloads as wl
-from gpu_util import (ORACLE_CODE, Guarded, assert_lse_close, assert_out_close, bits, packed_from_split, raw,
-                      sample_rows)
+from gpu_util import (HOST_THREADS, ORACLE_CODE, Guarded, assert_lse_close, assert_out_close, bits,
+                      compare_token_blocks, packed_from_split, raw)
 
 pytestmark = pytest.mark.gpu
 
@@ -150,7 +150,7 @@ def test_roundtrip_fp16(o):
 # ---- the bandwidth sweep -----------------------------------------------------------------
 SWEEP = wl.sweep()
 SWEEP_SMALL = [p for p in SWEEP if p.B == 512]
-SWEEP_LARGE = [p for p in SWEEP if p.B == 16384]
+SWEEP_LARGE = [p for p in SWEEP if p.B >= 4096]
 
 
 @pytest.mark.parametrize("w", SWEEP_SMALL, ids=lambda p: p.name)
@@ -161,28 +161,30 @@ def test_sweep_full_elementwise(o, w):
 
 
 @pytest.mark.parametrize("w", SWEEP_LARGE, ids=lambda p: p.name)
-def test_sweep_full_size_sampled(o, w):
-    """Full-size inputs; both entry points checked on sampled rows against the oracle, and
-    everywhere for finiteness (the inputs are finite and the LSEs never all -inf together)."""
+def test_sweep_full_size_elementwise(o, w):
+    """Full-size inputs of every B = 4096 and B = 16384 sweep point: every element of both
+    entry points against the oracle (run over token slices on all host cores).  The split
+    combine also returns the global LSE here, so that path is checked at full size too."""
     outputs, lses = wl.split_inputs(w)
     d_out, d_lse = outputs.cuda(), lses.cuda()
-    y = dcp.lse_weighted_combine(d_out, d_lse)
+    y, g = dcp.lse_weighted_combine(d_out, d_lse, return_lse=True)
     recv = torch.cat([d_out, d_lse.unsqueeze(-1).view(d_out.dtype)], dim=-1)
-    del d_out
+    del d_out, d_lse
     y2 = dcp.unpack_combine(recv)
     del recv
-    assert bool(torch.isfinite(y).all()) and bool(torch.isfinite(y2).all())
-    rows = sample_rows(w.B, w.Hr, 48, w.seed)
-    ref, _ = o.lse_combine_rows(raw(outputs), orc.BF16, raw(lses), rows)
-    bi = torch.tensor([r[0] for r in rows])
-    hi = torch.tensor([r[1] for r in rows])
-    assert_out_close(y.cpu()[bi, hi], ref, f"{w.name} combine (sampled)")
-    assert_out_close(y2.cpu()[bi, hi], ref, f"{w.name} unpack_combine (sampled)")
+    ro, rl = raw(outputs), raw(lses)
+
+    def ref(b0, b1):
+        return o.lse_combine_tokens(ro, orc.BF16, rl, b0, b1, return_lse=True, threads=HOST_THREADS)
+
+    compare_token_blocks(w.B, w.Hr * w.D, ref, [(y, "dcp_lse_combine"), (y2, "dcp_unpack_combine")],
+                         [(g, "dcp_lse_combine global lse")], w.name)
 
 
 def test_bench_step_full_size(o):
     """The bench's step at full size (largest sweep point): pack of cp_attn_out [B, N*Hr, D]
-    compared bit for bit everywhere, then unpack+combine of the send buffer on sampled rows."""
+    compared bit for bit everywhere, then every element of the unpack+combine of the send
+    buffer against the oracle's unpack+combine of the oracle's own send buffer."""
     w = wl.by_name("sweep_N16_B16384_D512")
     cp_out, cp_lse = wl.pack_inputs(w)
     send = dcp.pack(cp_out.cuda(), cp_lse.cuda(), w.N)
@@ -191,13 +193,13 @@ def test_bench_step_full_size(o):
     got_send = bits(send.cpu())
     assert np.array_equal(got_send, bits(ref_send)), "pack is not bit-exact"
     del got_send
-    y = dcp.unpack_combine(send, is_lse_base_on_e=w.is_lse_base_on_e)
-    rows = sample_rows(w.B, w.Hr, 48, 7)
-    ref, _ = o.unpack_combine_rows(ref_send, orc.BF16, w.D, rows)
-    bi = torch.tensor([r[0] for r in rows])
-    hi = torch.tensor([r[1] for r in rows])
-    assert_out_close(y.cpu()[bi, hi], ref, "bench step unpack_combine (sampled)")
-    assert bool(torch.isfinite(y).all())
+    y, g = dcp.unpack_combine(send, return_lse=True, is_lse_base_on_e=w.is_lse_base_on_e)
+
+    def ref(b0, b1):
+        return o.unpack_combine_tokens(ref_send, orc.BF16, w.D, b0, b1, return_lse=True, threads=HOST_THREADS)
+
+    compare_token_blocks(w.B, w.Hr * w.D, ref, [(y, "dcp_unpack_combine")], [(g, "dcp_unpack_combine lse")],
+                         "bench step")
 
 
 # ---- shapes, dtypes and edge cases -----------------------------------------------------------

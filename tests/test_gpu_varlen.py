@@ -14,7 +14,7 @@ import torch
 import decode_context_attention_dcp_b200 as dcp
 import oracle as orc
 from decode_context_attention_dcp_b200 import workloads as wl
-from gpu_util import ORACLE_CODE, assert_lse_close, assert_out_close, raw
+from gpu_util import HOST_THREADS, ORACLE_CODE, assert_lse_close, assert_out_close, compare_token_blocks, raw
 
 pytestmark = pytest.mark.gpu
 
@@ -143,36 +143,32 @@ def test_varlen_capacity_strided(o):
     assert_lse_close(g, rg, "capacity-strided varlen lse")
 
 
-def test_varlen_full_size_sampled(o):
+def test_varlen_full_size_elementwise(o):
     """The bench's largest combine shape (N=16, B=16384, H=16, D=512, bf16) with a decode batch of
-    short and long requests and padding, checked on sampled tokens: each sampled token is
-    rebuilt as a one-token request of its own and the oracle combines that sub-batch."""
+    short and long requests and padding: every element against the oracle (run over token
+    slices on all host cores).  The rows of shards without KV hold NaN and their LSEs 80."""
     N, B, H, D = 16, 16384, 16, 512
     w = wl.by_name("sweep_N16_B16384_D512")
     outputs, lses = wl.split_inputs(w)
     seq_lens, qsl = wl.decode_batch(wl.DecodeBatch(B=B, max_q=2, pad=300, p_short=0.4, short_max=N, max_seq=9000,
                                                    seed=45))
     mask = empty_mask(o, seq_lens, qsl, N, B, 1)
-    d_out, d_lse = outputs.cuda(), lses.cuda()
-    m = mask.cuda()
-    d_out[m] = float("nan")
-    d_lse[m] = 80.0
-    y, g = dcp.lse_weighted_combine_varlen(d_out, d_lse, seq_lens.cuda(), qsl.cuda(), return_lse=True)
+    outputs[mask] = float("nan")
+    lses[mask] = 80.0
+    y, g = dcp.lse_weighted_combine_varlen(outputs.cuda(), lses.cuda(), seq_lens.cuda(), qsl.cuda(),
+                                           return_lse=True)
     torch.cuda.synchronize()
     assert not bool(torch.isnan(y).any())
     pad0 = int(qsl[-1])
     assert bool((y[pad0:] == 0).all()) and bool(torch.isneginf(g[pad0:]).all())
-    rng = np.random.default_rng(45)
-    toks = np.sort(rng.choice(pad0, size=64, replace=False))
-    req = token_requests(qsl, B)
-    t = torch.from_numpy(toks)
-    s_out, s_lse = d_out[:, t].cpu(), d_lse[:, t].cpu()
-    s_seq = seq_lens[torch.from_numpy(req[toks])]
-    s_qsl = torch.arange(len(toks) + 1, dtype=torch.int32)
-    ry, rg = o.lse_combine_varlen(raw(s_out), orc.BF16, raw(s_lse), s_seq.numpy(), s_qsl.numpy(), return_lse=True)
-    t = t.cuda()
-    assert_out_close(y[t], ry, "full-size varlen (sampled)")
-    assert_lse_close(g[t], rg, "full-size varlen lse (sampled)")
+    ro, rl = raw(outputs), raw(lses)
+
+    def ref(b0, b1):
+        return o.lse_combine_varlen_tokens(ro, orc.BF16, rl, seq_lens.numpy(), qsl.numpy(), b0, b1,
+                                           return_lse=True, threads=HOST_THREADS)
+
+    compare_token_blocks(B, H * D, ref, [(y, "dcp_lse_combine_varlen")], [(g, "dcp_lse_combine_varlen lse")],
+                         "full-size varlen")
 
 
 def test_varlen_errors():
