@@ -69,6 +69,8 @@ def library() -> ctypes.CDLL:
                 lib.dcp_lse_pack_dim.restype = _i32
                 lib.dcp_pack.argtypes = [_ptr, _ptr, _ptr, _i64, _i64, _i64, _i32, _i32, _i64, _i64, _i64, _ptr]
                 lib.dcp_pack.restype = _i32
+                lib.dcp_testing_pack_stalled.argtypes = lib.dcp_pack.argtypes
+                lib.dcp_testing_pack_stalled.restype = _i32
                 lib.dcp_lse_combine.argtypes = [_ptr, _ptr, _ptr, _ptr, _i32, _i64, _i64, _i64, _i64, _i64, _i32,
                                                 _i32, _i32, _ptr]
                 lib.dcp_lse_combine.restype = _i32
@@ -100,8 +102,8 @@ def dcp_last_error() -> str:
 
 
 def dcp_wait_timeouts(reset: bool = False) -> int:
-    """Waits that timed out on the current device since the last reset (synchronises the
-    device).  Nonzero means some dcp_pack result is incomplete."""
+    """Pack CTAs whose wait for their copies timed out on the current device since the last
+    reset (synchronises the device).  Nonzero means some dcp_pack result is incomplete."""
     c = ctypes.c_uint64(0)
     _check(library().dcp_wait_timeouts(ctypes.byref(c), int(bool(reset))))
     return int(c.value)
@@ -157,7 +159,11 @@ def dcp_lse_pack_dim(dtype: torch.dtype) -> int:
 
 def dcp_pack(cp_attn_out: torch.Tensor, cp_attn_lse: torch.Tensor, send_buf: torch.Tensor, world_size: int,
              stream=None) -> None:
-    """cp_attn_out [B, H, D] + cp_attn_lse [B, H] fp32 -> send_buf [world_size, B, H/world_size, D + P]."""
+    """cp_attn_out [B, H, D] + cp_attn_lse [B, H] fp32 -> send_buf [world_size, B, H/world_size, D + P].
+
+    Asynchronous: the kernel's bounded waits for its copies cannot report to this call.  If one
+    ran out (never, while the copies work), send_buf is incomplete and dcp_wait_timeouts()
+    (which synchronises) is nonzero; callers that must be sure read it before trusting send_buf."""
     dev = _cuda(cp_attn_out, cp_attn_lse, send_buf)
     B, H, D = cp_attn_out.shape
     if cp_attn_lse.shape != (B, H) or cp_attn_lse.dtype != torch.float32:

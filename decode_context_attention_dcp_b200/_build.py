@@ -11,6 +11,7 @@ from __future__ import annotations
 import argparse
 import concurrent.futures
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -41,11 +42,28 @@ def inputs() -> list[str]:
     return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + sorted(glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
+def source_digest() -> str:
+    """SHA-256 of every input's bytes and of the compiler flags: a library built from other
+    sources (or a pushed library newer than its sources) is rebuilt, whatever the mtimes say."""
+    h = hashlib.sha256()
+    h.update(" ".join(ARCH + COMPILE_FLAGS + LINK_FLAGS).encode())
+    for p in inputs():
+        h.update(b"\0" + os.path.relpath(p, ROOT).encode() + b"\0")
+        with open(p, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def _digest_file(lib: str) -> str:
+    return lib + ".sha256"
+
+
 def stale(lib: str = LIBRARY) -> bool:
-    if not os.path.exists(lib):
+    """True unless ``lib`` exists and was built from exactly the current sources and flags."""
+    if not os.path.exists(lib) or not os.path.exists(_digest_file(lib)):
         return True
-    t = os.path.getmtime(lib)
-    return any(os.path.getmtime(p) > t for p in inputs())
+    with open(_digest_file(lib)) as fh:
+        return fh.read().strip() != source_digest()
 
 
 def _run(cmd: list[str]) -> None:
@@ -75,7 +93,11 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if verbose:
             for c in compiles + [link]:
                 print(" ".join(c))
+        digest = source_digest()
         os.replace(tmp, LIBRARY)
+        with open(_digest_file(LIBRARY) + ".tmp", "w") as fh:
+            fh.write(digest + "\n")
+        os.replace(_digest_file(LIBRARY) + ".tmp", _digest_file(LIBRARY))
     finally:
         if os.path.exists(tmp):
             os.unlink(tmp)

@@ -12,6 +12,7 @@
 #include <atomic>
 
 #include "dcp_host.h"
+#include "dcp_testing.h"
 
 namespace dcp_host {
 
@@ -107,13 +108,17 @@ bool pack_smem_reserved() {
     return true;
 }
 
-// Resident pack CTAs per SM for a given dynamic shared-memory size (one cached entry).
+// Resident pack CTAs per SM of the current device for a given dynamic shared-memory size
+// (one cached entry per device).
 int pack_resident_ctas(size_t smem) {
-    static std::atomic<uint64_t> cache{0};  // (smem << 16) | ctas
-    const uint64_t c = cache.load(std::memory_order_relaxed);
+    static std::atomic<uint64_t> cache[64];  // per device: (smem << 16) | ctas
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return resident_ctas(dcp::pack_kernel<>, dcp::kPackThreads, smem);
+    const uint64_t c = cache[dev].load(std::memory_order_relaxed);
     if (c && (c >> 16) == smem) return (int)(c & 0xffff);
     const int n = resident_ctas(dcp::pack_kernel<>, dcp::kPackThreads, smem);
-    cache.store(((uint64_t)smem << 16) | (uint64_t)n, std::memory_order_relaxed);
+    cache[dev].store(((uint64_t)smem << 16) | (uint64_t)n, std::memory_order_relaxed);
     return n;
 }
 
@@ -377,10 +382,14 @@ int32_t dcp_unpack_combine(const void *recv_buf, void *result, float *global_lse
     return dispatch_dtype<true>(dtype, a, static_cast<cudaStream_t>(cuda_stream));
 }
 
-int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_buf, int64_t B, int64_t H, int64_t D,
-                 int32_t world_size, int32_t dtype, int64_t out_stride_b, int64_t out_stride_h, int64_t lse_stride_b,
-                 void *cuda_stream) {
-    const char *fn = "dcp_pack";
+}  // extern "C"
+
+namespace {
+
+// dcp_pack with the wait limit and the first-tile stall of the timeout check explicit.
+int32_t pack_impl(const char *fn, const void *cp_attn_out, const float *cp_attn_lse, void *send_buf, int64_t B,
+                  int64_t H, int64_t D, int32_t world_size, int32_t dtype, int64_t out_stride_b, int64_t out_stride_h,
+                  int64_t lse_stride_b, void *cuda_stream, uint64_t wait_limit_ns, uint32_t stall_bytes) {
     int32_t st = check_common(fn, dtype, world_size, B, H, D);
     if (st != DCP_OK) return st;
     if (H % world_size != 0)
@@ -424,6 +433,8 @@ int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_b
     a.per_rank_magic = magic64((uint64_t)(B * a.Hr));
     a.hr_magic = magic64((uint64_t)a.Hr);
     a.pitch_magic = (uint32_t)(((uint64_t(1) << 32) + (uint64_t)a.row_pitch_w - 1) / (uint64_t)a.row_pitch_w);
+    a.wait_limit_ns = wait_limit_ns;
+    a.stall_bytes = stall_bytes;
     const size_t smem = (size_t)dcp::kPackStages * a.stage_w * 4;
     if (!pack_smem_reserved()) return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory for the pack kernel", fn);
     const int per_sm = pack_resident_ctas(smem);
@@ -432,6 +443,25 @@ int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_b
     const int grid = (int)(tiles < cap ? tiles : cap);
     dcp::pack_kernel<><<<grid, dcp::kPackThreads, smem, static_cast<cudaStream_t>(cuda_stream)>>>(a);
     return launch_status(fn);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_buf, int64_t B, int64_t H, int64_t D,
+                 int32_t world_size, int32_t dtype, int64_t out_stride_b, int64_t out_stride_h, int64_t lse_stride_b,
+                 void *cuda_stream) {
+    return pack_impl("dcp_pack", cp_attn_out, cp_attn_lse, send_buf, B, H, D, world_size, dtype, out_stride_b,
+                     out_stride_h, lse_stride_b, cuda_stream, dcp::kWaitLimitNs, 0u);
+}
+
+int32_t dcp_testing_pack_stalled(const void *cp_attn_out, const float *cp_attn_lse, void *send_buf, int64_t B,
+                                 int64_t H, int64_t D, int32_t world_size, int32_t dtype, int64_t out_stride_b,
+                                 int64_t out_stride_h, int64_t lse_stride_b, void *cuda_stream) {
+    // 16 bytes that never arrive keep each CTA's first tile waiting until the 20 ms limit
+    return pack_impl("dcp_testing_pack_stalled", cp_attn_out, cp_attn_lse, send_buf, B, H, D, world_size, dtype,
+                     out_stride_b, out_stride_h, lse_stride_b, cuda_stream, 20000000ull, 16u);
 }
 
 }  // extern "C"

@@ -29,8 +29,7 @@ int32_t launch_status(const char *what);
 // Multiprocessor count of the current device (cached per device).
 int sm_count();
 
-// Resident CTAs per SM of one kernel instance (cached per instance; the pool's
-// devices are identical).
+// Resident CTAs per SM of one kernel instance on the current device.
 template <class K>
 int resident_ctas(K kernel, int threads, size_t smem) {
     int n = 0;
@@ -38,11 +37,11 @@ int resident_ctas(K kernel, int threads, size_t smem) {
     return n;
 }
 
-// Per kernel instance: dynamic shared-memory opt-in (once per device) and the
+// Per kernel instance and device: the dynamic shared-memory opt-in (once) and the
 // resident-CTA count for the last shared-memory size seen.
 struct InstanceCache {
     std::atomic<int> opted[64];
-    std::atomic<uint64_t> occupancy{0};  // (smem << 16) | ctas
+    std::atomic<uint64_t> occupancy[64];  // (smem << 16) | ctas
 };
 
 template <class K>
@@ -58,10 +57,12 @@ bool reserve_smem(K kernel, InstanceCache &ic, size_t max_bytes) {
 
 template <class K>
 int cached_resident_ctas(K kernel, InstanceCache &ic, int threads, size_t smem) {
-    const uint64_t c = ic.occupancy.load(std::memory_order_relaxed);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return resident_ctas(kernel, threads, smem);
+    const uint64_t c = ic.occupancy[dev].load(std::memory_order_relaxed);
     if (c && (c >> 16) == smem) return (int)(c & 0xffff);
     const int n = resident_ctas(kernel, threads, smem);
-    ic.occupancy.store(((uint64_t)smem << 16) | (uint64_t)n, std::memory_order_relaxed);
+    ic.occupancy[dev].store(((uint64_t)smem << 16) | (uint64_t)n, std::memory_order_relaxed);
     return n;
 }
 

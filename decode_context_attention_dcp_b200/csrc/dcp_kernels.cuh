@@ -173,7 +173,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
-// Waits that time out: counted here, read (and cleared) by the host with dcp_wait_timeouts.
+// Pack CTAs whose wait for a tile's copies timed out: counted here, read (and cleared) by
+// the host with dcp_wait_timeouts.
 // Internal to each translation unit: the pack kernel and dcp_wait_timeouts share one.
 static __device__ unsigned long long g_wait_timeouts = 0;
 
@@ -185,14 +186,14 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
-// Waits for the barrier's phase with the given parity; false when a second passes (or the
+// Waits for the barrier's phase with the given parity; false when limit_ns pass (or the
 // iteration cap is reached) first.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t spin = 0; spin < (1u << 26); ++spin) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (global_ns() - t0 > kWaitLimitNs) break;
+        if (global_ns() - t0 > limit_ns) break;
     }
     return false;
 }
@@ -821,6 +822,9 @@ struct PackArgs {
     int32_t row_pitch_w;      // data_w + 1: words per packed row
     int32_t tile_rows;        // packed rows per tile
     int32_t stage_w;          // words per shared-memory stage (a multiple of 4)
+    uint64_t wait_limit_ns;   // limit of each wait for a tile's copies (kWaitLimitNs)
+    uint32_t stall_bytes;     // added to the byte count a CTA's first tile waits for: 0, except
+                              // in the check of the timeout path (its wait then runs out)
 };
 
 // Stores one landed tile: packed rows [i0, i0 + nrows) form the send range of words
@@ -956,7 +960,7 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
         const int nrows = tile_rows_of(k);
         const int slot = (int)(k % kPackStages);
         uint32_t *stage = s_stage + slot * stage_w;
-        if (tid == 0) mbar_arrive_expect_tx(&s_full[slot], (uint32_t)nrows * row_bytes);
+        if (tid == 0) mbar_arrive_expect_tx(&s_full[slot], (uint32_t)nrows * row_bytes + (k == 0 ? a.stall_bytes : 0u));
         for (int r = tid; r < nrows; r += kPackThreads) {
             fence_proxy_async();
             bulk_copy_g2s(stage + r * data_w, src + s_row_src[slot][r], row_bytes, &s_full[slot]);
@@ -984,17 +988,21 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
         // for tile k + kPackStages while the copies are in flight
         if (k + kPackStages < my_tiles) fill_table(k + kPackStages);
         cp_async_wait<kPackStages - 1>();  // this thread's LSE copies of tile k have landed
-        // the rows of tile k; a wait that times out is counted, and the CTA waits once more
-        // (bounded) for the copies it has in flight, then stops
-        uint64_t *bar = &s_full[(int)(k % kPackStages)];
-        const uint32_t parity = (uint32_t)((k / kPackStages) & 1);
-        if (!mbar_wait_bounded(bar, parity)) {
-            atomicAdd(&g_wait_timeouts, 1ull);
+        // the rows of tile k
+        if (!mbar_wait_bounded(&s_full[(int)(k % kPackStages)], (uint32_t)((k / kPackStages) & 1), a.wait_limit_ns))
             s_abort = 1;
-        }
         __syncthreads();                   // ... and everyone else's (and the table)
         if (s_abort) {
-            mbar_wait_bounded(bar, parity);
+            // A wait ran out: the CTA is counted and stops, its tiles unwritten.  Copies of
+            // tiles k .. k + kPackStages - 1 may still be in flight into this CTA's shared
+            // memory, so thread 0 first waits (bounded) for each of those tiles, which keeps
+            // the CTA resident until they land; every thread waits for its own word copies.
+            if (tid == 0) {
+                atomicAdd(&g_wait_timeouts, 1ull);
+                for (int64_t kk = k; kk < k + kPackStages && kk < my_tiles; ++kk)
+                    mbar_wait_bounded(&s_full[(int)(kk % kPackStages)], (uint32_t)((kk / kPackStages) & 1),
+                                      a.wait_limit_ns);
+            }
             cp_async_wait<0>();
             return;
         }

@@ -114,7 +114,9 @@ int32_t dcp_lse_pack_dim(int32_t dtype);
  *
  * The kernel waits for its bulk copies with a time limit; a wait that runs out
  * (never, while the copies work) leaves this call's send_buf incomplete and
- * is counted by dcp_wait_timeouts.
+ * is counted by dcp_wait_timeouts, and the call still returns DCP_OK (it
+ * returns before the kernel runs).  A caller that must be sure of send_buf
+ * reads dcp_wait_timeouts (which synchronises) before trusting it.
  */
 int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_buf,
                  int64_t B, int64_t H, int64_t D, int32_t world_size, int32_t dtype,
@@ -188,8 +190,10 @@ int32_t dcp_lse_combine_strided(const void *outputs, const float *lses, void *re
  *
  * outputs, lses, result, global_lse, out_stride_n, lse_stride_n: as
  *             dcp_lse_combine.
- * seq_lens    [num_reqs] int32 DEVICE array: KV length of each request, >= 0
- *             (a value <= 0 means no shard holds KV).
+ * seq_lens    [num_reqs] int32 DEVICE array: KV length of each request.  Shard n
+ *             holds KV when its local length is positive (n * interleave <
+ *             seq_lens[r]); 0 and negative values are accepted and mean that no
+ *             shard holds KV of the request.
  * query_start_loc  [num_reqs + 1] int32 DEVICE array, non-decreasing: the first
  *             token of each request, then the end of the last one.  Values that
  *             are not non-decreasing give unspecified results but no access
@@ -254,12 +258,13 @@ int32_t dcp_unpack_combine(const void *recv_buf, void *result, float *global_lse
                            void *cuda_stream);
 
 /*
- * Waits that timed out on the current device since the last reset.  dcp_pack waits for
- * its bulk copies with a limit of about one second per wait; a wait that runs out is
- * counted here and the CTA stops, so the send buffer of that call is incomplete.  A
- * nonzero count therefore means a result is invalid (it never happens when the copies
- * work).  Synchronises the device (the counter is read from device memory); with reset
- * != 0 the counter is cleared afterwards.  Returns DCP_ERR_CUDA if the read fails.
+ * Pack CTAs whose wait timed out on the current device since the last reset.  dcp_pack
+ * waits for its bulk copies with a limit of one second per wait; when a wait runs out the
+ * CTA is counted here and stops (after waiting, bounded, for the copies it has issued), so
+ * the send buffer of that call is incomplete.  A nonzero count therefore means a result is
+ * invalid (it never happens when the copies work).  Synchronises the device (the counter is
+ * read from device memory); with reset != 0 the counter is cleared afterwards.  Returns
+ * DCP_ERR_CUDA if the read fails.
  */
 int32_t dcp_wait_timeouts(uint64_t *count, int32_t reset);
 
