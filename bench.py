@@ -63,6 +63,10 @@ def parse_args(argv=None):
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the JSON line: per-kernel GB/s on every workload, as a markdown table")
     ap.add_argument("--sweep-reps", type=int, default=20)
+    ap.add_argument("--points", default="",
+                    help="--sweep: comma-separated workload names to run (default: every workload)")
+    ap.add_argument("--kernels", default="",
+                    help="--sweep: comma-separated kernel rows to run, by exact name (default: all)")
     return ap.parse_args(argv)
 
 
@@ -333,7 +337,8 @@ def workload_config(w) -> dict:
 # ---- per-kernel sweep ------------------------------------------------------------------------
 def run_sweep(args) -> int:
     """Median device time of each entry point on every workload (L2 flushed before each timed
-    launch); prints a markdown table."""
+    launch); prints a markdown table.  --points and --kernels restrict the table; only the
+    buffers the selected rows use are allocated."""
     import torch
 
     import decode_context_attention_dcp_b200 as dcp
@@ -343,65 +348,99 @@ def run_sweep(args) -> int:
     peak, peak_src = load_peak()
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     points = [wl.TINY, wl.GQA, wl.MLA, wl.ROUNDTRIP, *wl.sweep()]
+    if args.points:
+        points = [wl.by_name(n) for n in args.points.split(",")]
+    wanted = [k for k in args.kernels.split(",") if k]
+    S = 4  # KV splits of the producer in the fused-pack rows
     print(f"| workload | N | B | Hr | D | dtype | kernel | bytes | us | GB/s | frac of {peak:.0f} ({peak_src}) |")
     print("|---|---|---|---|---|---|---|---|---|---|---|")
     for w in points:
-        outputs, lses = wl.split_inputs(w)
-        d_out, d_lse = outputs.cuda(), lses.cuda()
-        del outputs, lses
-        recv = torch.cat([d_out, d_lse.unsqueeze(-1).view(d_out.dtype) if w.elem_bytes == 2 else d_lse.unsqueeze(-1)],
-                         dim=-1)
-        cp_out = d_out.permute(1, 0, 2, 3).reshape(w.B, w.H, w.D).contiguous()
-        cp_lse = d_lse.permute(1, 0, 2).reshape(w.B, w.H).contiguous()
-        res = torch.empty((w.B, w.Hr, w.D), dtype=d_out.dtype, device="cuda")
-        gl = torch.empty((w.B, w.Hr), dtype=torch.float32, device="cuda")
-        send = torch.empty_like(recv)
-        kernels = [
-            ("dcp_lse_combine", w.combine_bytes(),
-             lambda: dcp.dcp_lse_combine(d_out, d_lse, res, gl, is_lse_base_on_e=w.is_lse_base_on_e,
-                                         return_lse=w.return_lse)),
-            ("dcp_unpack_combine", w.combine_bytes(),
-             lambda: dcp.dcp_unpack_combine(recv, res, gl, is_lse_base_on_e=w.is_lse_base_on_e,
-                                            return_lse=w.return_lse)),
-            ("dcp_pack", w.pack_bytes(), lambda: dcp.dcp_pack(cp_out, cp_lse, send, w.N)),
-        ]
-        if w.B >= 4096 or w is wl.MLA:
-            # the same shards received head-scattered, [N, Hr, B, D] (dcp_lse_combine_strided)
-            hm_out = d_out.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
-            hm_lse = d_lse.permute(0, 2, 1).contiguous().permute(0, 2, 1)
-            kernels.append(("dcp_lse_combine_strided[head-major]", w.combine_bytes(),
-                            lambda: dcp.dcp_lse_combine(hm_out, hm_lse, res, gl, is_lse_base_on_e=w.is_lse_base_on_e,
-                                                        return_lse=w.return_lse)))
-            # a decode batch in which about 30% of the requests are too short to reach every
-            # shard (dcp_lse_combine_varlen reads only the shards that hold KV)
-            seq_lens, qsl = wl.decode_batch(wl.DecodeBatch(B=w.B, p_short=0.3, short_max=w.N, seed=w.seed))
-            req_of = torch.repeat_interleave(torch.arange(len(seq_lens)), qsl[1:] - qsl[:-1])
-            held = torch.clamp(seq_lens.long(), 0, w.N)  # token interleave: min(N, seq) shards hold KV
-            shards_read = int(held[req_of].sum())
-            d_seq, d_qsl = seq_lens.cuda(), qsl.cuda()
-            kernels.append(("dcp_lse_combine_varlen", w.varlen_combine_bytes(shards_read, len(seq_lens)),
-                            lambda: dcp.dcp_lse_combine_varlen(d_out, d_lse, res, d_seq, d_qsl, gl,
-                                                               is_lse_base_on_e=w.is_lse_base_on_e,
-                                                               return_lse=w.return_lse)))
-        if w.B >= 4096 or w is wl.MLA:
-            # a producer with S = 4 KV splits per rank: its split merge fused with the pack
-            # (dcp_combine_pack) against the merge into [B, H, D] followed by dcp_pack
-            S = 4
-            gen = torch.Generator(device="cuda").manual_seed(w.seed)
-            parts = torch.randn((S, w.B, w.H, w.D), generator=gen, device="cuda").to(d_out.dtype)
-            part_lse = torch.rand((S, w.B, w.H), generator=gen, device="cuda") * 20.0
-            merged = torch.empty((w.B, w.H, w.D), dtype=d_out.dtype, device="cuda")
-            merged_lse = torch.empty((w.B, w.H), dtype=torch.float32, device="cuda")
-            row = w.D * w.elem_bytes + 4
-            fused_bytes = w.B * w.H * (S * row + row)
-            kernels.append((f"dcp_combine_pack[S={S}]", fused_bytes,
-                            lambda: dcp.dcp_combine_pack(parts, part_lse, send, w.N)))
+        big = w.B >= 4096 or w is wl.MLA
+        names = ["dcp_lse_combine", "dcp_unpack_combine", "dcp_pack"]
+        if big:
+            names += ["dcp_lse_combine_strided[head-major]", "dcp_lse_combine_varlen", f"dcp_combine_pack[S={S}]",
+                      f"dcp_lse_combine+dcp_pack[S={S}]"]
+        names = [n for n in names if not wanted or n in wanted]
+        if not names:
+            continue
+        buf: dict = {}
+
+        def get(key):
+            """The point's buffers, made on first use."""
+            if key in buf:
+                return buf[key]
+            if key in ("out", "lse"):
+                outputs, lses = wl.split_inputs(w)
+                buf["out"], buf["lse"] = outputs.cuda(), lses.cuda()
+            elif key == "recv":
+                d_out, d_lse = get("out"), get("lse")
+                slot = d_lse.unsqueeze(-1).view(d_out.dtype) if w.elem_bytes == 2 else d_lse.unsqueeze(-1)
+                buf[key] = torch.cat([d_out, slot], dim=-1)
+            elif key == "cp":
+                buf[key] = (get("out").permute(1, 0, 2, 3).reshape(w.B, w.H, w.D).contiguous(),
+                            get("lse").permute(1, 0, 2).reshape(w.B, w.H).contiguous())
+            elif key == "res":
+                buf[key] = (torch.empty((w.B, w.Hr, w.D), dtype=wl.torch_dtype(w.dtype), device="cuda"),
+                            torch.empty((w.B, w.Hr), dtype=torch.float32, device="cuda"))
+            elif key == "send":
+                buf[key] = torch.empty((w.N, w.B, w.Hr, w.W), dtype=wl.torch_dtype(w.dtype), device="cuda")
+            elif key == "hm":
+                # the same shards received head-scattered, [N, Hr, B, D] (dcp_lse_combine_strided)
+                buf[key] = (get("out").permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3),
+                            get("lse").permute(0, 2, 1).contiguous().permute(0, 2, 1))
+            elif key == "varlen":
+                # a decode batch in which about 30% of the requests are too short to reach every
+                # shard (dcp_lse_combine_varlen reads only the shards that hold KV)
+                seq_lens, qsl = wl.decode_batch(wl.DecodeBatch(B=w.B, p_short=0.3, short_max=w.N, seed=w.seed))
+                req_of = torch.repeat_interleave(torch.arange(len(seq_lens)), qsl[1:] - qsl[:-1])
+                held = torch.clamp(seq_lens.long(), 0, w.N)  # token interleave: min(N, seq) shards hold KV
+                buf[key] = (seq_lens.cuda(), qsl.cuda(), int(held[req_of].sum()), len(seq_lens))
+            elif key == "parts":
+                # a producer with S KV splits per rank (its partials drawn on the device)
+                gen = torch.Generator(device="cuda").manual_seed(w.seed)
+                dt = wl.torch_dtype(w.dtype)
+                buf[key] = (torch.randn((S, w.B, w.H, w.D), generator=gen, device="cuda").to(dt),
+                            torch.rand((S, w.B, w.H), generator=gen, device="cuda") * 20.0)
+            elif key == "merged":
+                buf[key] = (torch.empty((w.B, w.H, w.D), dtype=wl.torch_dtype(w.dtype), device="cuda"),
+                            torch.empty((w.B, w.H), dtype=torch.float32, device="cuda"))
+            return buf[key]
+
+        row = w.D * w.elem_bytes + 4
+        fused_bytes = w.B * w.H * (S * row + row)
+
+        def make(name):
+            """(algorithmic bytes, launch) of one kernel row."""
+            kw = dict(is_lse_base_on_e=w.is_lse_base_on_e, return_lse=w.return_lse)
+            if name == "dcp_lse_combine":
+                d_out, d_lse, (res, gl) = get("out"), get("lse"), get("res")
+                return w.combine_bytes(), lambda: dcp.dcp_lse_combine(d_out, d_lse, res, gl, **kw)
+            if name == "dcp_unpack_combine":
+                recv, (res, gl) = get("recv"), get("res")
+                return w.combine_bytes(), lambda: dcp.dcp_unpack_combine(recv, res, gl, **kw)
+            if name == "dcp_pack":
+                (cp_out, cp_lse), send = get("cp"), get("send")
+                return w.pack_bytes(), lambda: dcp.dcp_pack(cp_out, cp_lse, send, w.N)
+            if name.startswith("dcp_lse_combine_strided"):
+                (hm_out, hm_lse), (res, gl) = get("hm"), get("res")
+                return w.combine_bytes(), lambda: dcp.dcp_lse_combine(hm_out, hm_lse, res, gl, **kw)
+            if name == "dcp_lse_combine_varlen":
+                d_out, d_lse, (res, gl) = get("out"), get("lse"), get("res")
+                d_seq, d_qsl, shards_read, reqs = get("varlen")
+                return (w.varlen_combine_bytes(shards_read, reqs),
+                        lambda: dcp.dcp_lse_combine_varlen(d_out, d_lse, res, d_seq, d_qsl, gl, **kw))
+            (parts, part_lse), send = get("parts"), get("send")
+            if name.startswith("dcp_combine_pack"):
+                return fused_bytes, lambda: dcp.dcp_combine_pack(parts, part_lse, send, w.N)
+            merged, merged_lse = get("merged")
 
             def two_step():
                 dcp.dcp_lse_combine(parts, part_lse, merged, merged_lse, return_lse=True)
                 dcp.dcp_pack(merged, merged_lse, send, w.N)
-            kernels.append((f"dcp_lse_combine+dcp_pack[S={S}]", fused_bytes + 2 * w.B * w.H * row, two_step))
-        for name, nbytes, fn in kernels:
+            return fused_bytes + 2 * w.B * w.H * row, two_step
+
+        for name in names:
+            nbytes, fn = make(name)
             for _ in range(3):
                 fn()
             times = []
@@ -419,8 +458,7 @@ def run_sweep(args) -> int:
             gbs = nbytes / (t * 1e-3) / 1e9
             print(f"| {w.name} | {w.N} | {w.B} | {w.Hr} | {w.D} | {w.dtype} | {name} | {nbytes} | {t * 1e3:.1f} | "
                   f"{gbs:.0f} | {gbs / peak:.3f} |", flush=True)
-        del d_out, d_lse, recv, cp_out, cp_lse, res, gl, send, kernels
-        parts = part_lse = merged = merged_lse = None
+        buf.clear()
         torch.cuda.empty_cache()
     return 0
 
