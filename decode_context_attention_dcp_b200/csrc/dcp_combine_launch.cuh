@@ -57,25 +57,85 @@ int32_t launch_g(dcp::CombineArgs a, int G, int cpl, cudaStream_t stream) {
 // covers a row, the sums are realigned once per output chunk ("uniform");
 // otherwise every shard's chunk is realigned, and that path keeps at least two
 // slots per lane.
+struct CombineShape {
+    int G;    // lanes per row
+    int cpl;  // chunk slots per lane per pass
+};
+
+inline CombineShape combine_shape(bool packed, bool uniform, int N, int chunks) {
+    int cpl_target = N >= 8 ? 1 : N >= 4 ? 2 : 4;
+    if (packed && !uniform && cpl_target < 2) cpl_target = 2;
+    // split layout, 8 or more shards, rows of at most 256 bytes: two chunk slots per lane
+    // (four rows per warp) measured 3-6% faster than one with 8-15 shards, 2% with 16
+    if (!packed && N >= 8 && chunks <= 16) cpl_target = 2;
+    const int per_lane = (chunks + cpl_target - 1) / cpl_target;
+    int G = 4;
+    while (G < per_lane && G < 32) G *= 2;
+    const int slots = (chunks + G - 1) / G;
+    return {G, slots >= 3 ? 4 : slots};  // one pass whenever slots <= 4
+}
+
+// The fused pack's 4-row group kernel: packed rows of D' = 32 C data words, C = 2 or 4, with
+// heads per rank a multiple of 4.  Tasks are 4-row groups, one per warp at a time.
+template <class K>
+int32_t launch_group(K kernel, InstanceCache &ic, const dcp::CombineArgs &a, size_t smem, const char *fn,
+                     cudaStream_t stream) {
+    if (!reserve_smem(kernel, ic, smem)) return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
+    const int per_sm = cached_resident_ctas(kernel, ic, dcp::kCombineThreads, smem);
+    constexpr int kWarps = dcp::kCombineThreads / 32;
+    const int64_t groups = (a.units + 3) / 4;
+    const int64_t want = (groups + kWarps - 1) / kWarps;
+    const int64_t cap = (int64_t)sm_count() * per_sm;
+    const int grid = (int)(want < cap ? want : cap);
+    kernel<<<grid, dcp::kCombineThreads, smem, stream>>>(a);
+    return launch_status(fn);
+}
+
+template <class T, int C, int NB, int MIN_CTAS>
+int32_t launch_group_pack(const dcp::CombineArgs &a, cudaStream_t stream) {
+    if (a.data_w != 32 * C || a.pack_hr % 4 != 0) return fail(DCP_ERR_INVALID_ARG, "dcp_combine_pack: internal shape error");
+    static InstanceCache ic;
+    if (!reserve_smem(dcp::group_pack_kernel<T, C, NB, MIN_CTAS>, ic,
+                      dcp::group_pack_smem_bytes(DCP_MAX_SHARDS, 32 * C)))
+        return fail(DCP_ERR_CUDA, "dcp_combine_pack: cannot reserve shared memory");
+    return launch_group(dcp::group_pack_kernel<T, C, NB, MIN_CTAS>, ic, a, dcp::group_pack_smem_bytes(a.N, a.data_w),
+                        "dcp_combine_pack", stream);
+}
+
+// NB = 2 splits in flight: measured best or equal for S = 4 and 8 (D' = 64: 0.89-0.94 of the
+// measured peak at B = 16384, against 0.75-0.81 for the per-row packed stores).
+template <class T>
+int32_t dispatch_group_pack(const dcp::CombineArgs &a, cudaStream_t stream) {
+    switch (a.data_w) {
+        case 64: return launch_group_pack<T, 2, 2, 3>(a, stream);
+        case 128: return launch_group_pack<T, 4, 2, 3>(a, stream);
+        default: return fail(DCP_ERR_INVALID_ARG, "dcp_combine_pack: internal shape error");
+    }
+}
+
 template <class T, bool PACKED>
 int32_t dispatch_combine(dcp::CombineArgs a, cudaStream_t stream) {
     const int chunks = a.chunks;
     const bool uniform = PACKED && (a.N == 1 || a.shard_stride_w % 4 == 0) && chunks <= 4 * 32;
-    int cpl_target = a.N >= 8 ? 1 : a.N >= 4 ? 2 : 4;
-    if (PACKED && !uniform && cpl_target < 2) cpl_target = 2;
-    // split layout, 8-15 shards, rows of at most 256 bytes: two chunk slots per lane (four
-    // rows per warp) measured 3-6% faster than one; packed rows lose with more slots
-    if (!PACKED && a.N >= 8 && a.N < 16 && chunks <= 16) cpl_target = 2;
-    const int per_lane = (chunks + cpl_target - 1) / cpl_target;
-    int G = 4;
-    while (G < per_lane && G < 32) G *= 2;
+    // the fused pack's group kernel: D' = 64 or 128 (at 32 the per-row path measured faster)
+    const bool group_rows = a.data_w == 64 || a.data_w == 128;
+    const CombineShape sh = combine_shape(PACKED, uniform, a.N, chunks);
+    const int G = sh.G, cpl = sh.cpl;
     a.slots = (chunks + G - 1) / G;
-    const int cpl = a.slots >= 3 ? 4 : a.slots;  // one pass whenever slots <= 4
     // Phase 1's reads one task ahead: measured worth it where phase 1's latency is exposed
     // (two shards, or packed rows of 1 KiB and more), and 2-4% slower where the stream
     // already hides it.
     const bool prefetch = a.N <= 2 || (PACKED && chunks >= 64);
     if constexpr (PACKED) {
+        if (uniform && chunks <= 16 && a.N >= 8) {
+            // rows of at most 256 bytes and 8 or more shards: four rows per warp (G = 8, two
+            // chunk slots per lane) with 8 shards' loads in flight (D = 128, B = 16384: 0.85-0.86
+            // of the measured peak at N = 8 against 0.79 with G = 16); at 16 or more shards,
+            // phase 1's reads one task ahead as well
+            a.slots = (chunks + 7) / 8;
+            if (a.N >= 16) return launch_combine<T, 8, 2, 8, true, 2, true, false, false, true>(a, stream);
+            return launch_combine<T, 8, 2, 8, true, 2, true, false, false, false>(a, stream);
+        }
         if (uniform) {
             if (prefetch) return launch_g<T, true, true, false, false, true>(a, G, cpl, stream);
             return launch_g<T, true, true, false, false, false>(a, G, cpl, stream);
@@ -83,7 +143,14 @@ int32_t dispatch_combine(dcp::CombineArgs a, cudaStream_t stream) {
         return launch_g<T, true, false, false, false, false>(a, G, cpl, stream);
     } else {
         if (a.varlen) return launch_g<T, false, false, true, false, true>(a, G, cpl, stream);
-        if (a.pack_b > 0) return launch_g<T, false, false, false, true, false>(a, G, cpl, stream);
+        if (a.pack_b > 0) {
+            if (group_rows && a.pack_hr % 4 == 0) {
+                // the weights summed as the split combine would (same lanes per row)
+                a.red_lanes = G;
+                return dispatch_group_pack<T>(a, stream);
+            }
+            return launch_g<T, false, false, false, true, false>(a, G, cpl, stream);
+        }
         if (prefetch) return launch_g<T, false, false, false, false, true>(a, G, cpl, stream);
         return launch_g<T, false, false, false, false, false>(a, G, cpl, stream);
     }

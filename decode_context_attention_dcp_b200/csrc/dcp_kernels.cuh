@@ -271,6 +271,7 @@ struct CombineArgs {
     int64_t pack_b;
     int64_t pack_hr;
     uint64_t pack_hr_magic;  // ceil(2^64 / pack_hr), 0 when pack_hr == 1
+    int32_t red_lanes;       // group_pack_kernel: lanes that reduce one row's LSEs (4, 8, 16, 32)
     int32_t varlen;
     int32_t num_reqs;
     int32_t interleave;
@@ -797,6 +798,155 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
         if constexpr (PREFETCH) buf ^= 1;
     }
     if constexpr (PREFETCH) cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
+// split merge written as 4-row groups of packed send rows (dcp_combine_pack, D' = 32 C,
+// C = 1, 2, 4, heads per rank a multiple of 4)
+//
+// Packed rows [4 g, 4 g + 4) of the send buffer [ranks, B, Hr, D' + 1] are 4 consecutive
+// heads of one (rank, token), i.e. the consecutive input rows u0 .. u0 + 3 of the split
+// partials, and one aligned span of D' + 1 chunks of the send buffer.  A warp merges one
+// group at a time.  Lane l = 8 r + j loads chunks j + 8 k (k < C) of input row r, so each
+// load instruction reads 128 consecutive bytes of every row (split rows are aligned).
+// Phase 1 reduces each row's S LSEs over `red_lanes` lanes (the split combine's grouping, so
+// that the weights, hence the bits, equal those of dcp_lse_combine), phase 2 runs fp32 FMAs
+// over the splits with NB splits in flight.  The rounded words and the merged LSEs are placed
+// in a copy of the span in shared memory (row r at word r (D' + 1)), from which lane l stores
+// chunks l + 32 k, and lane 31 the span's last chunk: 16-byte stores of 512 consecutive bytes,
+// every word of the span written once.
+__host__ __device__ constexpr size_t group_pack_smem_bytes(int N, int data_w) {
+    // per warp: the span copy (4 (D' + 1) words) and the weights [N][4] floats
+    return (size_t)(kCombineThreads / 32) * (4 * (data_w + 1) + N * 4) * 4;
+}
+
+template <class T, int C, int NB, int MIN_CTAS>
+__global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) group_pack_kernel(const CombineArgs a) {
+    constexpr int kE = T::kPerWord;
+    constexpr int kWarps = kCombineThreads / 32;
+    extern __shared__ uint4 s_dyn[];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int N = a.N;
+    const int data_w = a.data_w;  // 32 C
+    const int pitch = data_w + 1;
+    const int span_w = 4 * pitch;  // a multiple of 4
+    uint32_t *s_span = reinterpret_cast<uint32_t *>(s_dyn) + (size_t)warp * span_w;
+    float *sw = reinterpret_cast<float *>(s_dyn) + (size_t)kWarps * span_w + (size_t)warp * N * 4;
+    __shared__ uint32_t s_glse_all[kWarps][4];
+    uint32_t *s_glse = s_glse_all[warp];
+    const int r = lane >> 3;  // the input row of this lane in phase 2
+    const int j = lane & 7;
+    const uint32_t *lses = reinterpret_cast<const uint32_t *>(a.lses);
+    const int64_t per_rank = a.pack_b * a.pack_hr;
+    const int64_t groups = (a.units + 3) >> 2;  // units = ranks * B * Hr packed rows, a multiple of 4
+
+    for (int64_t g = (int64_t)blockIdx.x * kWarps + warp; g < groups; g += (int64_t)gridDim.x * kWarps) {
+        const int64_t p0 = g * 4;
+        const int64_t rank = p0 / per_rank;
+        const int64_t rem = p0 - rank * per_rank;
+        const int64_t b = rem / a.pack_hr;
+        const int64_t u0 = b * a.heads + rank * a.pack_hr + (rem - b * a.pack_hr);
+        const int64_t row = (u0 + r) * data_w + 4 * j;  // this lane's first input word in split 0
+        Words<4> x[NB][C];
+        auto issue = [&](int n0) {
+#pragma unroll
+            for (int i = 0; i < NB; ++i)
+#pragma unroll
+                for (int k = 0; k < C; ++k) {
+                    if (n0 + i < N) {
+                        x[i][k] = load_stream<4>(a.src + (int64_t)(n0 + i) * a.shard_stride_w + row + 32 * k);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) x[i][k].w[e] = 0u;
+                    }
+                }
+        };
+        issue(0);
+
+        // ---- phase 1: weights of each row over the splits ---------------------------------------
+        // `red` lanes per row, 32 / red rows per pass: the lane grouping of the split combine
+        // for the same S and D', so that the weights are summed in the same order and the
+        // result equals dcp_lse_combine + dcp_pack bit for bit.
+        // (any other value is taken as 8, so that every loop below ends whatever the argument)
+        const int red = (a.red_lanes == 4 || a.red_lanes == 16 || a.red_lanes == 32) ? a.red_lanes : 8;
+        for (int rb = 0; rb < 4; rb += 32 / red) {
+            const int rr = rb + lane / red;  // >= 4 on idle lanes (red = 4)
+            const int jj = lane % red;
+            const bool act = rr < 4;
+            float lmax = -INFINITY;
+            for (int n = jj; act && n < N; n += red) {
+                const float l = sanitize_lse(load_word(lses + (int64_t)n * a.lse_stride_n + u0 + rr));
+                sw[n * 4 + rr] = l;
+                lmax = fmaxf(lmax, l);
+            }
+            for (int o = red / 2; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+            const float m = (lmax == -INFINITY) ? 0.0f : lmax;
+            float wsum = 0.0f;
+            for (int n = jj; act && n < N; n += red) {
+                const float x1 = sw[n * 4 + rr] - m;
+                float w = a.base_e ? expf(x1) : exp2f(x1);
+                if (w != w) w = 0.0f;
+                sw[n * 4 + rr] = w;
+                wsum += w;
+            }
+            for (int o = red / 2; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+            const float denom = fmaxf(wsum, 1e-10f);
+            for (int n = jj; act && n < N; n += red) sw[n * 4 + rr] = sw[n * 4 + rr] / denom;
+            if (act && jj == 0) s_glse[rr] = __float_as_uint((a.base_e ? logf(wsum) : log2f(wsum)) + m);
+        }
+        __syncwarp();
+
+        // ---- phase 2: weighted sum over the splits --------------------------------------------
+        float acc[C][4][kE];
+#pragma unroll
+        for (int k = 0; k < C; ++k)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+                for (int h = 0; h < kE; ++h) acc[k][e][h] = 0.0f;
+        for (int n0 = 0; n0 < N; n0 += NB) {
+            if (n0 > 0) issue(n0);
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+                if (n0 + i >= N) break;  // the same for the whole warp
+                const float w = sw[(n0 + i) * 4 + r];
+#pragma unroll
+                for (int k = 0; k < C; ++k)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float f[kE];
+                        T::decode(x[i][k].w[e], f);
+#pragma unroll
+                        for (int h = 0; h < kE; ++h) acc[k][e][h] = fmaf(w, f[h], acc[k][e][h]);
+                    }
+            }
+        }
+        // the packed span in shared memory: row r's words at r (D' + 1), its LSE after them
+        uint32_t *srow = s_span + r * pitch + 4 * j;
+#pragma unroll
+        for (int k = 0; k < C; ++k)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) srow[32 * k + e] = T::encode(acc[k][e]);
+        if (j == 0) s_span[r * pitch + data_w] = s_glse[r];
+        __syncwarp();
+        uint32_t *span = a.result + p0 * pitch;
+        const uint4 *sv = reinterpret_cast<const uint4 *>(s_span);
+#pragma unroll
+        for (int k = 0; k < C; ++k) {
+            const uint4 v = sv[lane + 32 * k];
+            Words<4> o;
+            o.w[0] = v.x; o.w[1] = v.y; o.w[2] = v.z; o.w[3] = v.w;
+            store_words<4>(span + 4 * (lane + 32 * k), o);
+        }
+        if (lane == 31) {
+            const uint4 v = sv[32 * C];
+            Words<4> o;
+            o.w[0] = v.x; o.w[1] = v.y; o.w[2] = v.z; o.w[3] = v.w;
+            store_words<4>(span + 4 * 32 * C, o);
+        }
+        __syncwarp();  // shared memory is reused by the next group
+    }
 }
 
 // ---------------------------------------------------------------------------

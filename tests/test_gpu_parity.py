@@ -229,6 +229,22 @@ def test_edge_shapes(o, N, B, Hr, D, dtype):
         w, outputs, lses = _case(N, B, Hr, D, dtype, seed, base_e=base_e)
         check_split(o, w, outputs, lses, True)
         check_packed(o, w, packed_from_split(outputs, lses), True)
+    # the same into guarded outputs: nothing is written outside them
+    ry, rg = o.lse_combine(raw(outputs), ORACLE_CODE[outputs.dtype], raw(lses), return_lse=True,
+                           is_lse_base_on_e=False)
+    for packed in (False, True):
+        res = Guarded((B, Hr, D), outputs.dtype)
+        gl = Guarded((B, Hr), torch.float32)
+        if packed:
+            dcp.dcp_unpack_combine(packed_from_split(outputs, lses).cuda(), res.tensor, gl.tensor,
+                                   is_lse_base_on_e=False, return_lse=True)
+        else:
+            dcp.dcp_lse_combine(outputs.cuda(), lses.cuda(), res.tensor, gl.tensor, is_lse_base_on_e=False,
+                                return_lse=True)
+        res.check()
+        gl.check()
+        assert_out_close(res.tensor, ry, f"guarded packed={packed}")
+        assert_lse_close(gl.tensor, rg, f"guarded packed={packed}")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp16", "fp32"])
