@@ -346,7 +346,10 @@ def run_sweep(args) -> int:
 
     torch.cuda.set_device(0)
     peak, peak_src = load_peak()
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    # L2 is emptied before each timed launch by READING 512 MB (4x L2): the lines it leaves are
+    # clean, so nothing is written back to DRAM during the timed launch (a write-flush leaves up
+    # to an L2's worth of dirty lines whose write-back the timed launch would pay for)
+    flush = torch.zeros(128 << 20, dtype=torch.float32, device="cuda")
     points = [wl.TINY, wl.GQA, wl.MLA, wl.ROUNDTRIP, *wl.sweep()]
     if args.points:
         points = [wl.by_name(n) for n in args.points.split(",")]
@@ -447,7 +450,7 @@ def run_sweep(args) -> int:
             for _ in range(args.sweep_reps):
                 # the flush empties L2 and keeps the GPU busy while the host enqueues the timed
                 # launch, so host-side call overhead never lands between the two events
-                flush.zero_()
+                flush.sum()
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record()
                 fn()
