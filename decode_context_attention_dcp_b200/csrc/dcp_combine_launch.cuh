@@ -26,6 +26,23 @@ int32_t launch_combine(const dcp::CombineArgs &a, cudaStream_t stream) {
     return launch_status(fn);
 }
 
+// The single-pass packed combine (online_unpack_kernel), one pass per row.
+template <class T, int G, int CPL, int NB, int MIN_CTAS>
+int32_t launch_online(const dcp::CombineArgs &a, cudaStream_t stream) {
+    auto kernel = dcp::online_unpack_kernel<T, G, CPL, NB, MIN_CTAS>;
+    static InstanceCache ic;
+    if (a.slots > CPL) return fail(DCP_ERR_INVALID_ARG, "dcp_unpack_combine: internal shape error");
+    constexpr int kUnitsPerWarp = 32 / G;
+    constexpr int kWarps = dcp::kCombineThreads / 32;
+    const int per_sm = cached_resident_ctas(kernel, ic, dcp::kCombineThreads, 0);
+    const int64_t tasks = (a.units + kUnitsPerWarp - 1) / kUnitsPerWarp;
+    const int64_t want = (tasks + kWarps - 1) / kWarps;
+    const int64_t cap = (int64_t)sm_count() * per_sm;
+    const int grid = (int)(want < cap ? want : cap);
+    kernel<<<grid, dcp::kCombineThreads, 0, stream>>>(a);
+    return launch_status("dcp_unpack_combine");
+}
+
 // Occupancy: the kernel keeps NB * CPL 16-byte loads in flight per lane, so the
 // bytes in flight per SM are set by how many warps fit.  Capping registers so
 // that 3 CTAs fit (2 for the four-slot shapes, which spill otherwise) measured
@@ -127,14 +144,26 @@ int32_t dispatch_combine(dcp::CombineArgs a, cudaStream_t stream) {
     // already hides it.
     const bool prefetch = a.N <= 2 || (PACKED && chunks >= 64);
     if constexpr (PACKED) {
-        if (uniform && chunks <= 16 && a.N >= 8) {
-            // rows of at most 256 bytes and 8 or more shards: four rows per warp (G = 8, two
-            // chunk slots per lane) with 8 shards' loads in flight (D = 128, B = 16384: 0.85-0.86
-            // of the measured peak at N = 8 against 0.79 with G = 16); at 16 or more shards,
-            // phase 1's reads one task ahead as well
+        if (uniform && chunks <= 32 && a.N >= 3) {
+            // rows of at most 512 bytes and 3 or more shards: the single-pass kernel, whose LSEs
+            // come with each batch's data.  Measured at B = 16384 (fractions of the measured
+            // peak, single-pass against two-phase): D = 64 N = 8, 16: 0.91, 0.99 vs 0.74, 0.77;
+            // D = 128 N = 3, 4, 8, 16: 0.86, 0.96, 0.99, 1.03 vs 0.71, 0.77, 0.94, 0.91;
+            // D = 256 N = 4, 8: 0.96, 0.98 vs 0.82, 0.81.  At N = 2 the two kinds tie.
+            if (chunks <= 8) {
+                a.slots = (chunks + 3) / 4;
+                return launch_online<T, 4, 2, 4, 3>(a, stream);
+            }
+            if (chunks <= 16) {
+                if (a.N >= 8) {
+                    a.slots = (chunks + 7) / 8;
+                    return launch_online<T, 8, 2, 4, 3>(a, stream);
+                }
+                a.slots = (chunks + 3) / 4;
+                return launch_online<T, 4, 4, 4, 2>(a, stream);
+            }
             a.slots = (chunks + 7) / 8;
-            if (a.N >= 16) return launch_combine<T, 8, 2, 8, true, 2, true, false, false, true>(a, stream);
-            return launch_combine<T, 8, 2, 8, true, 2, true, false, false, false>(a, stream);
+            return launch_online<T, 8, 4, 4, 2>(a, stream);
         }
         if (uniform) {
             if (prefetch) return launch_g<T, true, true, false, false, true>(a, G, cpl, stream);

@@ -801,6 +801,168 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
 }
 
 // ---------------------------------------------------------------------------
+// single-pass unpack + combine of packed rows (uniform shard stride, one pass per row)
+//
+// The two-phase kernel must read every shard's LSE (the row's tail chunk) before it can weight
+// any data, and with the LSE inside the data stream that read is a DRAM round trip of its own
+// per task.  Here each batch of NB shards brings its LSEs with its data: lane j < NB of a row
+// also loads shard n0 + j's tail chunk, which holds the row's LSE (word q, q = the row's word
+// offset from a 16-byte boundary) and up to 3 of its last data words.  The combine rules are
+// applied to the running state (m, S, sums) batch by batch:
+//   l_n <- -inf if NaN or +-inf;  m' = max(m, max over the batch);
+//   c = exp(m - m') (1 while m' is still -inf);  w_n = exp(l_n - m'), NaN -> 0;
+//   S <- c S + sum w_n;  sums <- c sums + sum w_n o_n.
+// At the end the sums are divided by max(S, 1e-10) and the global LSE is ln S + m (log2 in
+// base 2; m taken as 0 when every LSE was -inf).  This is the page's arithmetic with the
+// weights formed against the running maximum and rescaled to the final one, so it differs from
+// the two-phase result by fp32 rounding only.  Row layout, realignment and stores are those of
+// combine_kernel's uniform packed path (G lanes per row, CPL chunk slots per lane).
+template <class T, int G, int CPL, int NB, int MIN_CTAS>
+__global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) online_unpack_kernel(const CombineArgs a) {
+    static_assert(NB <= G, "each shard of a batch needs a lane to read its tail chunk");
+    constexpr int kUnitsPerWarp = 32 / G;
+    constexpr int kWarps = kCombineThreads / 32;
+    constexpr int kE = 4 * T::kPerWord;
+    const int lane = threadIdx.x & 31;
+    const int ul = lane / G;
+    const int j = lane % G;
+    const int row_lane0 = lane - j;
+    const int next_lane = (lane & ~(G - 1)) | ((j + 1) & (G - 1));
+    const int64_t tasks = (a.units + kUnitsPerWarp - 1) / kUnitsPerWarp;
+    const bool base_e = a.base_e != 0;
+
+    for (int64_t task = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); task < tasks;
+         task += (int64_t)gridDim.x * kWarps) {
+        const int64_t u = task * kUnitsPerWarp + ul;
+        const bool valid = u < a.units;
+        const int64_t row = u * a.row_pitch_w;  // the row's first word in shard 0
+        const int q = (int)(row & 3);             // the same in every shard (uniform stride)
+        const int64_t wa0 = row - q;              // the row's aligned window in shard 0
+        int c[CPL];
+        bool act[CPL];
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+            c[k] = j + G * k;
+            act[k] = valid && c[k] < a.chunks;
+        }
+        Words<4> x[NB][CPL];
+        Words<4> t;  // lane j < NB: the tail chunk of shard n0 + j
+        auto issue = [&](int n0) {
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+                const int64_t wa = (int64_t)(n0 + i) * a.shard_stride_w + wa0;
+#pragma unroll
+                for (int k = 0; k < CPL; ++k) {
+                    if (n0 + i < a.N && act[k]) {
+                        x[i][k] = load_stream<4>(a.src + wa + 4 * c[k]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) x[i][k].w[e] = 0u;
+                    }
+                }
+            }
+            if (valid && j < NB && n0 + j < a.N) {
+                t = load_chunk_bounded(a.src, (int64_t)(n0 + j) * a.shard_stride_w + wa0 + 4 * (int64_t)a.chunks, a.total_w);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) t.w[e] = 0u;
+            }
+        };
+        issue(0);
+
+        float m = -INFINITY, S = 0.0f;
+        float acc[CPL][kE];
+#pragma unroll
+        for (int k = 0; k < CPL; ++k)
+#pragma unroll
+            for (int e = 0; e < kE; ++e) acc[k][e] = 0.0f;
+        float tacc[3 * T::kPerWord];  // this lane's shards: weighted sum of the tail chunks' first 3 words
+#pragma unroll
+        for (int e = 0; e < 3 * T::kPerWord; ++e) tacc[e] = 0.0f;
+
+        for (int n0 = 0; n0 < a.N; n0 += NB) {
+            if (n0 > 0) issue(n0);
+            // the batch's LSEs, its maximum and the rescaling of the running state
+            const bool mine = valid && j < NB && n0 + j < a.N;
+            const uint32_t lbits = q == 0 ? t.w[0] : q == 1 ? t.w[1] : q == 2 ? t.w[2] : t.w[3];
+            const float l = mine ? sanitize_lse(lbits) : -INFINITY;
+            const float bmax = group_max<G>(l);
+            const float mn = fmaxf(m, bmax);
+            const float scale = mn == -INFINITY ? 1.0f : (base_e ? expf(m - mn) : exp2f(m - mn));
+            float w = base_e ? expf(l - mn) : exp2f(l - mn);
+            if (w != w) w = 0.0f;
+            if (!mine) w = 0.0f;
+            m = mn;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                for (int e = 0; e < kE; ++e) acc[k][e] *= scale;
+            {
+                const uint32_t tw[3] = {t.w[0], t.w[1], t.w[2]};
+#pragma unroll
+                for (int e = 0; e < 3; ++e) {
+                    float f[T::kPerWord];
+                    T::decode(tw[e], f);
+#pragma unroll
+                    for (int h = 0; h < T::kPerWord; ++h)
+                        tacc[e * T::kPerWord + h] = fmaf(w, f[h], tacc[e * T::kPerWord + h] * scale);
+                }
+            }
+            S *= scale;
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+                if (n0 + i >= a.N) break;  // the same for the whole warp
+                const float wi = __shfl_sync(0xffffffffu, w, row_lane0 + i);
+                S += wi;
+#pragma unroll
+                for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float f[T::kPerWord];
+                        T::decode(x[i][k].w[e], f);
+#pragma unroll
+                        for (int h = 0; h < T::kPerWord; ++h)
+                            acc[k][e * T::kPerWord + h] = fmaf(wi, f[h], acc[k][e * T::kPerWord + h]);
+                    }
+            }
+        }
+        // normalise by the clamped sum; the tail sums over the row's lanes
+        const float r = 1.0f / fmaxf(S, 1e-10f);
+#pragma unroll
+        for (int e = 0; e < 3 * T::kPerWord; ++e) tacc[e] = group_sum<G>(tacc[e]) * r;
+        if (a.return_lse && valid && j == 0) a.glse[u] = (base_e ? logf(S) : log2f(S)) + (m == -INFINITY ? 0.0f : m);
+        // round, then realign: result chunk c = words q.. of sums c and c + 1 (the next lane's, lane
+        // 0's next slot for lane G - 1, the tail sums for the row's last chunk)
+        Words<4> enc[CPL];
+#pragma unroll
+        for (int k = 0; k < CPL; ++k)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float f[T::kPerWord];
+#pragma unroll
+                for (int h = 0; h < T::kPerWord; ++h) f[h] = acc[k][e * T::kPerWord + h] * r;
+                enc[k].w[e] = T::encode(f);
+            }
+        Words<4> tenc;
+#pragma unroll
+        for (int e = 0; e < 3; ++e) tenc.w[e] = T::encode(&tacc[e * T::kPerWord]);
+        tenc.w[3] = 0u;
+        uint32_t *res = a.result + u * a.data_w;
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+            Words<4> send = enc[k];
+            if (k + 1 < CPL && j == 0) send = enc[k + 1 < CPL ? k + 1 : k];
+            Words<4> nx;
+#pragma unroll
+            for (int e = 0; e < 3; ++e) nx.w[e] = __shfl_sync(0xffffffffu, send.w[e], next_lane);
+            nx.w[3] = 0u;
+            if (act[k] && c[k] == a.chunks - 1) nx = tenc;
+            if (act[k]) store_words<4>(res + 4 * (int64_t)c[k], funnel_words(enc[k], nx, q));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // split merge written as 4-row groups of packed send rows (dcp_combine_pack, D' = 32 C,
 // C = 1, 2, 4, heads per rank a multiple of 4)
 //
