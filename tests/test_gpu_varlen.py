@@ -85,10 +85,11 @@ def test_varlen_matches_oracle(o, dtype, N, interleave, max_q):
     assert bool(torch.isinf(g[int(qsl[-1]):]).all())  # padding slots
 
 
-def test_varlen_with_every_shard_full_is_the_plain_combine(o):
-    """Requests whose KV reaches every shard and no padding: the same launch arithmetic as
-    dcp_lse_combine, so the results are identical bit for bit."""
-    N, B, H, D = 8, 200, 8, 256
+@pytest.mark.parametrize("N,D", [(8, 256), (8, 128), (16, 128), (4, 128), (3, 512)])
+def test_varlen_with_every_shard_full_is_the_plain_combine(o, N, D):
+    """Requests whose KV reaches every shard and no padding: the same lanes per row as
+    dcp_lse_combine, so the weights are summed alike and the results are identical bit for bit."""
+    B, H = 200, 8
     w = wl.CombineWorkload("varlen_full", N=N, B=B, Hr=H, D=D, lse_lo=-5.0, lse_hi=15.0, p_neginf=0.1,
                            p_nan=0.02, seed=41)
     outputs, lses = [t.cuda() for t in wl.split_inputs(w)]
