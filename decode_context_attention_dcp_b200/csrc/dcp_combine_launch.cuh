@@ -130,67 +130,157 @@ int32_t dispatch_group_pack(const dcp::CombineArgs &a, cudaStream_t stream) {
     }
 }
 
-template <class T, bool PACKED>
-int32_t dispatch_combine(dcp::CombineArgs a, cudaStream_t stream) {
+// The packed receive layout (dcp_unpack_combine).
+template <class T>
+int32_t dispatch_packed(dcp::CombineArgs a, cudaStream_t stream) {
     const int chunks = a.chunks;
-    const bool uniform = PACKED && (a.N == 1 || a.shard_stride_w % 4 == 0) && chunks <= 4 * 32;
-    // the fused pack's group kernel: D' = 64 or 128 (at 32 the per-row path measured faster)
-    const bool group_rows = a.data_w == 64 || a.data_w == 128;
-    const CombineShape sh = combine_shape(PACKED, uniform, a.N, chunks);
+    const bool uniform = (a.N == 1 || a.shard_stride_w % 4 == 0) && chunks <= 4 * 32;
+    const CombineShape sh = combine_shape(true, uniform, a.N, chunks);
     const int G = sh.G, cpl = sh.cpl;
     a.slots = (chunks + G - 1) / G;
     // Phase 1's reads one task ahead: measured worth it where phase 1's latency is exposed
     // (two shards, or packed rows of 1 KiB and more), and 2-4% slower where the stream
     // already hides it.
-    const bool prefetch = a.N <= 2 || (PACKED && chunks >= 64);
-    if constexpr (PACKED) {
-        if (uniform && chunks <= 32 && a.N >= 3) {
-            // rows of at most 512 bytes and 3 or more shards: the single-pass kernel, whose LSEs
-            // come with each batch's data.  Measured at B = 16384 (fractions of the measured
-            // peak, single-pass against two-phase): D = 64 N = 8, 16: 0.91, 0.99 vs 0.74, 0.77;
-            // D = 128 N = 3, 4, 8, 16: 0.86, 0.96, 0.99, 1.03 vs 0.71, 0.77, 0.94, 0.91;
-            // D = 256 N = 4, 8: 0.96, 0.98 vs 0.82, 0.81.  At N = 2 the two kinds tie.
-            if (chunks <= 8) {
-                a.slots = (chunks + 3) / 4;
-                return launch_online<T, 4, 2, 4, 3>(a, stream);
-            }
-            if (chunks <= 16) {
-                if (a.N >= 8) {
-                    a.slots = (chunks + 7) / 8;
-                    return launch_online<T, 8, 2, 4, 3>(a, stream);
-                }
-                a.slots = (chunks + 3) / 4;
-                return launch_online<T, 4, 4, 4, 2>(a, stream);
-            }
-            a.slots = (chunks + 7) / 8;
-            return launch_online<T, 8, 4, 4, 2>(a, stream);
+    const bool prefetch = a.N <= 2 || chunks >= 64;
+    if (uniform && chunks <= 32 && a.N >= 3) {
+        // rows of at most 512 bytes and 3 or more shards: the single-pass kernel, whose LSEs
+        // come with each batch's data.  Measured at B = 16384 (fractions of the measured
+        // peak, single-pass against two-phase): D = 64 N = 8, 16: 0.91, 0.99 vs 0.74, 0.77;
+        // D = 128 N = 3, 4, 8, 16: 0.86, 0.96, 0.99, 1.03 vs 0.71, 0.77, 0.94, 0.91;
+        // D = 256 N = 4, 8: 0.96, 0.98 vs 0.82, 0.81.  At N = 2 the two kinds tie.
+        if (chunks <= 8) {
+            a.slots = (chunks + 3) / 4;
+            return launch_online<T, 4, 2, 4, 3>(a, stream);
         }
-        if (uniform) {
-            if (prefetch) return launch_g<T, true, true, false, false, true>(a, G, cpl, stream);
-            return launch_g<T, true, true, false, false, false>(a, G, cpl, stream);
-        }
-        return launch_g<T, true, false, false, false, false>(a, G, cpl, stream);
-    } else {
-        if (a.varlen) {
-            if (G == 8 && chunks > 8 && chunks <= 16 && a.N >= 8) {
-                // the plain combine's shape (G = 8, so the weights are summed alike) with all 8
-                // shards of a batch in flight: D = 128, B = 16384, N = 8 / 16 took 1.09 / 1.03 of the
-                // plain combine's time per byte read, against 1.11 / 1.05 with 4
-                return launch_combine<T, 8, 2, 8, false, 2, false, true, false, true>(a, stream);
+        if (chunks <= 16) {
+            if (a.N >= 8) {
+                a.slots = (chunks + 7) / 8;
+                return launch_online<T, 8, 2, 4, 3>(a, stream);
             }
-            return launch_g<T, false, false, true, false, true>(a, G, cpl, stream);
+            a.slots = (chunks + 3) / 4;
+            return launch_online<T, 4, 4, 4, 2>(a, stream);
         }
-        if (a.pack_b > 0) {
-            if (group_rows && a.pack_hr % 4 == 0) {
-                // the weights summed as the split combine would (same lanes per row)
-                a.red_lanes = G;
-                return dispatch_group_pack<T>(a, stream);
-            }
-            return launch_g<T, false, false, false, true, false>(a, G, cpl, stream);
-        }
-        if (prefetch) return launch_g<T, false, false, false, false, true>(a, G, cpl, stream);
-        return launch_g<T, false, false, false, false, false>(a, G, cpl, stream);
+        a.slots = (chunks + 7) / 8;
+        return launch_online<T, 8, 4, 4, 2>(a, stream);
     }
+    if (uniform) {
+        if (prefetch) return launch_g<T, true, true, false, false, true>(a, G, cpl, stream);
+        return launch_g<T, true, true, false, false, false>(a, G, cpl, stream);
+    }
+    return launch_g<T, true, false, false, false, false>(a, G, cpl, stream);
+}
+
+// Shape of the split-layout combine (dcp_lse_combine and its strided, variable-length and
+// fused-pack forms).  Lanes per row G: the row's chunks over about 2 slots per lane with 8
+// or more shards (one pass, CPL = 2, 4 shards per batch; rows of at most 8 chunks with 16 or
+// more shards: one slot, 8 shards per batch), about 4 with 4-7 shards and 8 with fewer
+// (passes of CPL = 4, 2 shards per batch, or all 3).  Phase 1's LSE words are copied one
+// task ahead wherever there are fewer than 8 shards or rows of at most 256 bytes.  Measured
+// on B200 (split bf16, B = 16384, 16 heads; fractions of the measured copy peak, this shape
+// against the previous one):
+//   D = 64:  N = 3, 6, 32: 0.89, 1.01, 1.04 against 0.84, 0.84, 0.92
+//   D = 128: N = 3, 4, 8, 12: 1.07, 1.06, 1.09, 1.08 against 0.86, 0.94, 1.06, 1.03
+//   D = 256: N = 3, 8, 12: 1.03, 1.04, 1.06 against 0.91, 0.94, 0.95
+//   D = 512: N = 2, 4: 1.00, 1.04 against 0.98, 1.01
+// and within 2% of the best of 22 shapes at every other N in 2-32.  Only G decides the
+// result bits (the lanes that sum a row's weights); CPL and the batch only order the loads.
+struct SplitShape {
+    int G;          // lanes per row
+    int cpl;        // chunk slots per lane per pass: 1, 2 or 4
+    int nb;         // shards per batch: cpl * nb 16-byte loads in flight per lane
+    bool prefetch;  // phase 1's LSE words copied into shared memory one task ahead
+};
+
+inline SplitShape split_shape(int N, int chunks) {
+    const int per_lane = (N >= 16 && chunks <= 8) ? 1 : N >= 8 ? 2 : N >= 4 ? 4 : 8;
+    int G = 4;
+    while (G * per_lane < chunks && G < 32) G *= 2;
+    const int slots = (chunks + G - 1) / G;
+    const int cpl = slots <= 2 ? slots : N >= 8 ? 2 : 4;
+    const int nb = cpl == 1 ? 8 : cpl == 2 ? (N <= 2 ? 2 : 4) : (N == 3 ? 4 : 2);
+    return {G, cpl, nb, N < 8 || chunks <= 16};
+}
+
+// The variable-length combine's shape.  A row whose request reaches only some shards issues
+// fewer loads in the same time, so with 4 or more shards each lane keeps 16 loads in flight:
+// G = about a quarter of the row's chunks, 4 slots of 4 shards.  The weights must be summed as
+// the plain combine sums them (so that a batch whose requests reach every shard gives the
+// same bits): lane j of G sums shards j, j + G, ... and the G lanes then reduce by halves, so
+// two lane counts agree whenever N <= 2 * the smaller one; otherwise the plain shape is
+// kept, as it is with fewer than 4 shards.  Measured at B = 16384, split bf16, time against
+// the plain combine's time scaled by the bytes read (about 30% of the requests reaching only
+// some shards), this shape against the plain one:
+//   D = 128, N = 4, 8: 1.11, 1.07 against 1.18, 1.10
+//   D = 256, N = 4, 8, 16: 1.04, 1.04, 1.04 against 1.11, 1.09, 1.05
+//   D = 512, N = 4, 8, 16: 1.03, 1.05, 1.03 against 1.08, 1.08, 1.03
+inline SplitShape varlen_shape(int N, int chunks, const SplitShape &plain) {
+    if (N < 4) return plain;
+    int G = 4;
+    while (G * 4 < chunks && G < 32) G *= 2;
+    const int lo = G < plain.G ? G : plain.G;
+    if (G != plain.G && N > 2 * lo) return plain;
+    const int slots = (chunks + G - 1) / G;
+    const int cpl = slots <= 2 ? slots : 4;
+    return {G, cpl, cpl == 1 ? 8 : 4, true};
+}
+
+// Registers are capped so that 3 CTAs fit (8 loads in flight per lane), 4 for the 4-load
+// shape and 2 for the four-slot shapes, which spill otherwise.  Single-slot shapes only
+// arise with G = 4 or 8 and the 2 x 2 shape with G = 4 (rows of at most 8 chunks); a shape
+// with a G it does not arise with takes the two-slot instance, which computes the same
+// result.
+template <class T, int G, bool VARLEN, bool PACK_OUT, bool PREFETCH>
+int32_t launch_split_g(const dcp::CombineArgs &a, const SplitShape &s, cudaStream_t stream) {
+    if (s.cpl == 4) {
+        if (s.nb == 4) return launch_combine<T, G, 4, 4, false, 2, false, VARLEN, PACK_OUT, PREFETCH>(a, stream);
+        return launch_combine<T, G, 4, 2, false, 2, false, VARLEN, PACK_OUT, PREFETCH>(a, stream);
+    }
+    if constexpr (G <= 8) {
+        if (s.cpl == 1) return launch_combine<T, G, 1, 8, false, 3, false, VARLEN, PACK_OUT, PREFETCH>(a, stream);
+    }
+    if constexpr (G == 4) {
+        if (s.nb == 2) return launch_combine<T, 4, 2, 2, false, 4, false, VARLEN, PACK_OUT, PREFETCH>(a, stream);
+    }
+    return launch_combine<T, G, 2, 4, false, 3, false, VARLEN, PACK_OUT, PREFETCH>(a, stream);
+}
+
+template <class T, bool VARLEN, bool PACK_OUT, bool PREFETCH>
+int32_t launch_split(const dcp::CombineArgs &a, const SplitShape &s, cudaStream_t stream) {
+    switch (s.G) {
+        case 4: return launch_split_g<T, 4, VARLEN, PACK_OUT, PREFETCH>(a, s, stream);
+        case 8: return launch_split_g<T, 8, VARLEN, PACK_OUT, PREFETCH>(a, s, stream);
+        case 16: return launch_split_g<T, 16, VARLEN, PACK_OUT, PREFETCH>(a, s, stream);
+        default: return launch_split_g<T, 32, VARLEN, PACK_OUT, PREFETCH>(a, s, stream);
+    }
+}
+
+// The split layout: dcp_lse_combine, dcp_lse_combine_strided, dcp_lse_combine_varlen and
+// dcp_combine_pack.
+template <class T>
+int32_t dispatch_split(dcp::CombineArgs a, cudaStream_t stream) {
+    const SplitShape s = split_shape(a.N, a.chunks);
+    a.slots = (a.chunks + s.G - 1) / s.G;
+    if (a.varlen) {
+        const SplitShape v = varlen_shape(a.N, a.chunks, s);
+        a.slots = (a.chunks + v.G - 1) / v.G;
+        if (v.G == 8 && v.cpl == 2 && a.chunks > 8 && a.chunks <= 16 && a.N >= 8) {
+            // all 8 shards of a batch in flight: D = 128, B = 16384, N = 16 took 1.03 of the
+            // plain combine's time per byte read, against 1.05 with 4
+            return launch_combine<T, 8, 2, 8, false, 2, false, true, false, true>(a, stream);
+        }
+        return launch_split<T, true, false, true>(a, v, stream);
+    }
+    if (a.pack_b > 0) {
+        // the fused pack's group kernel: D' = 64 or 128 (at 32 the per-row path measured faster)
+        if ((a.data_w == 64 || a.data_w == 128) && a.pack_hr % 4 == 0) {
+            a.red_lanes = s.G;  // the weights summed as the split combine would (same lanes per row)
+            return dispatch_group_pack<T>(a, stream);
+        }
+        if (s.prefetch) return launch_split<T, false, true, true>(a, s, stream);
+        return launch_split<T, false, true, false>(a, s, stream);
+    }
+    if (s.prefetch) return launch_split<T, false, false, true>(a, s, stream);
+    return launch_split<T, false, false, false>(a, s, stream);
 }
 
 }  // namespace dcp_host

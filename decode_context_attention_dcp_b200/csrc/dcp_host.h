@@ -72,5 +72,9 @@ int cached_resident_ctas(K kernel, InstanceCache &ic, int threads, size_t smem) 
 int32_t dispatch_combine_bf16(const dcp::CombineArgs &a, bool packed, cudaStream_t stream);
 int32_t dispatch_combine_fp16(const dcp::CombineArgs &a, bool packed, cudaStream_t stream);
 int32_t dispatch_combine_fp32(const dcp::CombineArgs &a, bool packed, cudaStream_t stream);
+// The split-layout half of each (its own translation unit).
+int32_t dispatch_split_bf16(const dcp::CombineArgs &a, cudaStream_t stream);
+int32_t dispatch_split_fp16(const dcp::CombineArgs &a, cudaStream_t stream);
+int32_t dispatch_split_fp32(const dcp::CombineArgs &a, cudaStream_t stream);
 
 }  // namespace dcp_host

@@ -85,19 +85,24 @@ def test_varlen_matches_oracle(o, dtype, N, interleave, max_q):
     assert bool(torch.isinf(g[int(qsl[-1]):]).all())  # padding slots
 
 
-@pytest.mark.parametrize("N,D", [(8, 256), (8, 128), (16, 128), (4, 128), (3, 512)])
-def test_varlen_with_every_shard_full_is_the_plain_combine(o, N, D):
-    """Requests whose KV reaches every shard and no padding: the same lanes per row as
-    dcp_lse_combine, so the weights are summed alike and the results are identical bit for bit."""
+@pytest.mark.parametrize("N,D,dtype", [(8, 256, "bf16"), (8, 128, "bf16"), (16, 128, "bf16"), (4, 128, "bf16"),
+                                       (3, 512, "bf16"), (4, 512, "bf16"), (8, 512, "bf16"), (16, 256, "bf16"),
+                                       (32, 256, "bf16"), (33, 512, "bf16"), (64, 128, "bf16"), (16, 64, "bf16"),
+                                       (8, 64, "bf16"), (8, 128, "fp32"), (5, 96, "fp16"), (2, 128, "bf16")])
+def test_varlen_with_every_shard_full_is_the_plain_combine(o, N, D, dtype):
+    """Requests whose KV reaches every shard and no padding: the weights are summed as
+    dcp_lse_combine sums them (the same lanes per row, or lane counts that agree for this
+    shard count), so the results are identical bit for bit."""
     B, H = 200, 8
-    w = wl.CombineWorkload("varlen_full", N=N, B=B, Hr=H, D=D, lse_lo=-5.0, lse_hi=15.0, p_neginf=0.1,
-                           p_nan=0.02, seed=41)
+    w = wl.CombineWorkload("varlen_full", N=N, B=B, Hr=H, D=D, dtype=dtype, lse_lo=-5.0, lse_hi=15.0,
+                           p_neginf=0.1, p_nan=0.02, seed=41)
     outputs, lses = [t.cuda() for t in wl.split_inputs(w)]
     seq_lens, qsl = wl.decode_batch(wl.DecodeBatch(B=B, max_q=2, p_short=0.0, short_max=N, max_seq=5000,
                                                    seed=41))
     y, g = dcp.lse_weighted_combine_varlen(outputs, lses, seq_lens.cuda(), qsl.cuda(), return_lse=True)
     yp, gp = dcp.lse_weighted_combine(outputs, lses, return_lse=True)
-    assert torch.equal(y.view(torch.int16), yp.view(torch.int16))
+    word = torch.int32 if y.element_size() == 4 else torch.int16
+    assert torch.equal(y.view(word), yp.view(word))
     assert torch.equal(g.view(torch.int32), gp.view(torch.int32))
 
 
