@@ -94,34 +94,66 @@ uint64_t magic64(uint64_t d) {
 
 // The pack kernel's dynamic shared memory can exceed the default 48 KiB: opt in
 // once per device, for the largest stage any accepted row width needs.
-bool pack_smem_reserved() {
-    static std::atomic<int> done[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    if (dev < 64 && done[dev].load(std::memory_order_acquire)) return true;
+// One pack kernel instance: its dynamic shared memory is reserved once per device (enough for
+// a stage of `max_stage_w` words), and its resident CTAs per SM are cached per device for the
+// last dynamic shared-memory size asked.
+template <int STAGES, int MAX_ROWS>
+struct PackInstance {
+    static constexpr auto kernel = dcp::pack_kernel<STAGES, dcp::kPackThreads, MAX_ROWS>;
+    static bool reserve(int max_stage_w) {
+        static std::atomic<int> done[64];
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return false;
+        if (dev < 64 && done[dev].load(std::memory_order_acquire)) return true;
+        const size_t bytes = (size_t)STAGES * max_stage_w * 4;
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+            return false;
+        if (dev < 64) done[dev].store(1, std::memory_order_release);
+        return true;
+    }
+    static int resident(size_t smem) {
+        static std::atomic<uint64_t> cache[64];  // per device: (smem << 16) | ctas
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+            return resident_ctas(kernel, dcp::kPackThreads, smem);
+        const uint64_t c = cache[dev].load(std::memory_order_relaxed);
+        if (c && (c >> 16) == smem) return (int)(c & 0xffff);
+        const int n = resident_ctas(kernel, dcp::kPackThreads, smem);
+        cache[dev].store(((uint64_t)smem << 16) | (uint64_t)n, std::memory_order_relaxed);
+        return n;
+    }
+};
+
+// Tile geometry and launch of one pack instance.  A stage holds about `stage_words` words of
+// source rows (at least one row, at most MAX_ROWS) and their LSE words, plus 4 words of slack
+// for the second aligned read of the last chunk.
+template <int STAGES, int MAX_ROWS>
+int32_t launch_pack(const char *fn, dcp::PackArgs a, int stage_words, bool runs_if_short, cudaStream_t stream) {
+    using I = PackInstance<STAGES, MAX_ROWS>;
+    a.tile_rows = (stage_words - 8) / a.row_pitch_w;
+    if (a.tile_rows < 1) a.tile_rows = 1;
+    if (a.tile_rows > MAX_ROWS) a.tile_rows = MAX_ROWS;
+    a.stage_w = ((a.tile_rows * a.row_pitch_w + 3) & ~3) + 4;
     const int max_stage_w = (int)(((kMaxD + 1 + 3) & ~int64_t(3)) + 4);  // one fp32 row of kMaxD words
-    const size_t bytes = (size_t)dcp::kPackStages * max_stage_w * 4;
-    if (cudaFuncSetAttribute(dcp::pack_kernel<>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
-        cudaSuccess)
-        return false;
-    if (dev < 64) done[dev].store(1, std::memory_order_release);
-    return true;
+    if (!I::reserve(stage_words + 8 > max_stage_w ? stage_words + 8 : max_stage_w))
+        return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory for the pack kernel", fn);
+    const size_t smem = (size_t)STAGES * a.stage_w * 4;
+    const int per_sm = I::resident(smem);
+    const int64_t tiles = (a.rows + a.tile_rows - 1) / a.tile_rows;
+    const int64_t cap = (int64_t)sm_count() * per_sm;
+    // With contiguous heads, the rows of one (rank, token) can be copied as one run.  Measured
+    // on B200 (bf16, fraction of the measured copy peak): runs win for launches of at most
+    // ~24 tiles per CTA (N = 8, B = 1024, D = 512: 0.91 against 0.85; N = 2, B = 16384,
+    // D = 128: 0.88 against 0.80) and with rows of at most 128 bytes (D = 64: 0.84 against
+    // 0.57), and lose in longer launches of larger rows, where one copy per row keeps more
+    // copies in flight (N = 16, B = 16384: D = 512 0.94 against 0.87, D = 128 0.91 against 0.85).
+    const bool contiguous = a.src_stride_h_w == a.data_w;
+    const bool runs = contiguous && (!runs_if_short || tiles <= 24 * cap);
+    a.max_run = runs ? (int32_t)(a.Hr < (int64_t(1) << 20) ? a.Hr : (int64_t(1) << 20)) : 1;
+    const int grid = (int)(tiles < cap ? tiles : cap);
+    I::kernel<<<grid, dcp::kPackThreads, smem, stream>>>(a);
+    return launch_status(fn);
 }
-
-// Resident pack CTAs per SM of the current device for a given dynamic shared-memory size
-// (one cached entry per device).
-int pack_resident_ctas(size_t smem) {
-    static std::atomic<uint64_t> cache[64];  // per device: (smem << 16) | ctas
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        return resident_ctas(dcp::pack_kernel<>, dcp::kPackThreads, smem);
-    const uint64_t c = cache[dev].load(std::memory_order_relaxed);
-    if (c && (c >> 16) == smem) return (int)(c & 0xffff);
-    const int n = resident_ctas(dcp::pack_kernel<>, dcp::kPackThreads, smem);
-    cache[dev].store(((uint64_t)smem << 16) | (uint64_t)n, std::memory_order_relaxed);
-    return n;
-}
-
 
 template <bool PACKED>
 int32_t dispatch_dtype(int32_t dtype, const dcp::CombineArgs &a, cudaStream_t stream) {
@@ -422,12 +454,6 @@ int32_t pack_impl(const char *fn, const void *cp_attn_out, const float *cp_attn_
     a.lse_stride_b = lse_stride_b;
     a.data_w = (int32_t)(D * es / 4);
     a.row_pitch_w = a.data_w + 1;
-    // a stage holds about 16 KiB of source rows (at least one) and their LSE
-    // words, plus 4 words of slack for the second aligned read of the last chunk
-    a.tile_rows = (dcp::kPackMinStageWords - 8) / a.row_pitch_w;
-    if (a.tile_rows < 1) a.tile_rows = 1;
-    if (a.tile_rows > dcp::kPackMaxTileRows) a.tile_rows = dcp::kPackMaxTileRows;
-    a.stage_w = ((a.tile_rows * a.row_pitch_w + 3) & ~3) + 4;
     if (a.rows >= (int64_t(1) << 32))
         return fail(DCP_ERR_INVALID_ARG, "%s: more than 2^32 packed rows", fn);
     a.per_rank_magic = magic64((uint64_t)(B * a.Hr));
@@ -435,14 +461,13 @@ int32_t pack_impl(const char *fn, const void *cp_attn_out, const float *cp_attn_
     a.pitch_magic = (uint32_t)(((uint64_t(1) << 32) + (uint64_t)a.row_pitch_w - 1) / (uint64_t)a.row_pitch_w);
     a.wait_limit_ns = wait_limit_ns;
     a.stall_bytes = stall_bytes;
-    const size_t smem = (size_t)dcp::kPackStages * a.stage_w * 4;
-    if (!pack_smem_reserved()) return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory for the pack kernel", fn);
-    const int per_sm = pack_resident_ctas(smem);
-    const int64_t tiles = (a.rows + a.tile_rows - 1) / a.tile_rows;
-    const int64_t cap = (int64_t)sm_count() * per_sm;
-    const int grid = (int)(tiles < cap ? tiles : cap);
-    dcp::pack_kernel<><<<grid, dcp::kPackThreads, smem, static_cast<cudaStream_t>(cuda_stream)>>>(a);
-    return launch_status(fn);
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    // Rows of at most 128 bytes: 2 stages of up to 256 rows (about 32 KiB), copied as runs
+    // (D = 64: 0.84 of peak, against 0.72 for 3 stages of 64 rows with runs).  Otherwise 3
+    // stages of up to 64 rows or 32 KiB (measured best among 2-6 stages of 16-48 KiB and 64-256
+    // rows, which need the smaller stages' 4 CTAs per SM at D = 128).
+    if (a.data_w <= 32) return launch_pack<2, 256>(fn, a, 12288, false, stream);
+    return launch_pack<dcp::kPackStages, dcp::kPackMaxTileRows>(fn, a, dcp::kPackMinStageWords, true, stream);
 }
 
 }  // namespace

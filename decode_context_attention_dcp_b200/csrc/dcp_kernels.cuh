@@ -1134,6 +1134,8 @@ struct PackArgs {
     int32_t row_pitch_w;      // data_w + 1: words per packed row
     int32_t tile_rows;        // packed rows per tile
     int32_t stage_w;          // words per shared-memory stage (a multiple of 4)
+    int32_t max_run;          // rows per bulk copy, at most: 1, or more when the heads of a token
+                              // are contiguous (src_stride_h_w == data_w)
     uint64_t wait_limit_ns;   // limit of each wait for a tile's copies (kWaitLimitNs)
     uint32_t stall_bytes;     // added to the byte count a CTA's first tile waits for: 0, except
                               // in the check of the timeout path (its wait then runs out)
@@ -1223,14 +1225,16 @@ __device__ __forceinline__ void pack_store_tile(const uint32_t *stage, uint32_t 
 //   the row's LSE word (rows are >= 5 words, so a chunk holds at most one LSE).
 //   The partial chunks at the two ends of the range use 4-byte stores.
 // Every word of the send buffer is written once, by one CTA.
-template <int STAGES = kPackStages, int THREADS = kPackThreads>
+template <int STAGES = kPackStages, int THREADS = kPackThreads, int MAX_ROWS = kPackMaxTileRows>
 __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
     constexpr int kPackStages = STAGES;
     constexpr int kPackThreads = THREADS;
+    constexpr int kPackMaxTileRows = MAX_ROWS;
     extern __shared__ uint4 s_stage_v4[];
     uint32_t *s_stage = reinterpret_cast<uint32_t *>(s_stage_v4);
     __shared__ int64_t s_row_src[kPackStages][kPackMaxTileRows];  // word offset of each source row
     __shared__ int64_t s_row_lse[kPackStages][kPackMaxTileRows];  // index of each row's LSE
+    __shared__ int32_t s_row_run[kPackStages][kPackMaxTileRows];  // rows copied from this row on (0: none)
     __shared__ uint64_t s_full[kPackStages];                      // a stage's rows have landed
     __shared__ int s_abort;                                       // a wait timed out
     const int tid = threadIdx.x;
@@ -1260,13 +1264,25 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
             const uint64_t rank = div_magic(i, a.per_rank_magic);
             const uint64_t rem = i - rank * (uint64_t)(a.B * a.Hr);
             const uint64_t b = div_magic(rem, a.hr_magic);
-            const uint64_t head = rank * (uint64_t)a.Hr + (rem - b * (uint64_t)a.Hr);
+            const uint64_t hh = rem - b * (uint64_t)a.Hr;  // head within the rank
+            const uint64_t head = rank * (uint64_t)a.Hr + hh;
             s_row_src[slot][r] = (int64_t)b * a.src_stride_b_w + (int64_t)head * a.src_stride_h_w;
             s_row_lse[slot][r] = (int64_t)b * a.lse_stride_b + (int64_t)head;
+            // with contiguous heads, rows r .. r + run - 1 (heads hh .. of this rank and token b,
+            // up to the next multiple of max_run and within the tile) are one run of source
+            // words, copied by the run's first row
+            int run = 1;
+            if (a.max_run > 1) {
+                const int pos = (int)(hh % (uint64_t)a.max_run);
+                run = (r == 0 || pos == 0)
+                          ? (int)min(min((int64_t)(a.max_run - pos), (int64_t)a.Hr - (int64_t)hh), (int64_t)(nrows - r))
+                          : 0;
+            }
+            s_row_run[slot][r] = run;
         }
     };
-    // each source row is one bulk copy (16-byte aligned, a multiple of 16 bytes) that
-    // completes on the stage's barrier; the LSE words are 4-byte cp.async copies
+    // each run of source rows is one bulk copy (16-byte aligned, a multiple of 16 bytes)
+    // that completes on the stage's barrier; the LSE words are 4-byte cp.async copies
     const uint32_t row_bytes = (uint32_t)data_w * 4u;
     auto issue = [&](int64_t k) {
         const int nrows = tile_rows_of(k);
@@ -1274,8 +1290,11 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
         uint32_t *stage = s_stage + slot * stage_w;
         if (tid == 0) mbar_arrive_expect_tx(&s_full[slot], (uint32_t)nrows * row_bytes + (k == 0 ? a.stall_bytes : 0u));
         for (int r = tid; r < nrows; r += kPackThreads) {
-            fence_proxy_async();
-            bulk_copy_g2s(stage + r * data_w, src + s_row_src[slot][r], row_bytes, &s_full[slot]);
+            const int run = s_row_run[slot][r];
+            if (run > 0) {
+                fence_proxy_async();
+                bulk_copy_g2s(stage + r * data_w, src + s_row_src[slot][r], (uint32_t)run * row_bytes, &s_full[slot]);
+            }
             cp_async_word(stage + lse_base + r, lse + s_row_lse[slot][r]);
         }
     };

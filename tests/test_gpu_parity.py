@@ -508,6 +508,34 @@ def test_pack_edge_shapes(o, B, H, D, ws, dtype):
     assert dcp.dcp_wait_timeouts() == 0
 
 
+PACK_RUNS = [  # B, H, D, world_size, dtype: contiguous heads
+    (5000, 42, 64, 6, "bf16"),    # 128-byte rows, 7 heads per rank: runs cut by 256-row tiles
+    (2000, 20, 32, 4, "fp32"),    # 128-byte fp32 rows
+    (700, 24, 16, 3, "fp16"),     # 32-byte rows
+    (64, 512, 128, 2, "bf16"),    # 256 heads per rank: runs longer than a 64-row tile
+    (33, 12, 520, 4, "bf16"),     # 1040-byte rows, tiles of 31 rows
+    (3000, 16, 512, 2, "bf16"),   # a short launch of 1 KiB rows
+    (301, 7, 8, 7, "bf16"), (97, 8, 4, 2, "fp32"), (3, 4, 8192, 2, "bf16")]
+
+
+@pytest.mark.parametrize("B,H,D,ws,dtype", PACK_RUNS)
+def test_pack_head_runs(o, B, H, D, ws, dtype):
+    """Contiguous heads, where a (rank, token)'s rows may be copied as one run: bit-exact
+    against the oracle, with guard bands around the send buffer."""
+    dt = wl.torch_dtype(dtype)
+    gen = torch.Generator().manual_seed(B * 7 + H * 3 + D)
+    out = torch.randn(B, H, D, generator=gen).to(dt)
+    lse = torch.randn(B, H, generator=gen)
+    lse.view(torch.int32)[0, 0] = 0x7FC0ABCD             # NaN payload must survive
+    P = dcp.dcp_lse_pack_dim(dt)
+    send = Guarded((ws, B, H // ws, D + P), dt)
+    dcp.dcp_pack(out.cuda(), lse.cuda(), send.tensor, ws)
+    send.check()
+    ref = o.pack(raw(out), raw(lse), ws, ORACLE_CODE[dt])
+    assert np.array_equal(bits(send.tensor.cpu()), bits(ref))
+    assert dcp.dcp_wait_timeouts() == 0
+
+
 def test_concurrent_host_threads(o):
     """Four host threads, each with its own stream and inputs, pack and combine at the same
     time (first calls included, which set up each kernel instance): every result matches the
