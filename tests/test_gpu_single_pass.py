@@ -89,3 +89,27 @@ def test_full_size_single_pass(o):
 
     compare_token_blocks(w.B, w.Hr * w.D, ref, [(y, "dcp_unpack_combine")], [(g, "dcp_unpack_combine lse")],
                          "single pass full size")
+
+
+@pytest.mark.parametrize("dtype,D", [("bf16", 512), ("fp16", 512), ("fp32", 256), ("bf16", 264), ("bf16", 320)])
+@pytest.mark.parametrize("N", [3, 4, 5, 8, 15, 16])
+def test_wide_rows_quarter_lanes(o, dtype, D, N):
+    """Packed rows of 513 bytes to 1 KiB with 3-15 shards take the two-phase kernel with 16
+    lanes per row (16 shards: 32 lanes); the same special rows as above, against the oracle.
+    12 tokens of 3 heads keep every shard's stride a multiple of 16 bytes."""
+    B, Hr = 12, 3
+    w = wl.CombineWorkload(f"wide_N{N}_D{D}_{dtype}", N=N, B=B, Hr=Hr, D=D, dtype=dtype, lse_lo=-20.0,
+                           lse_hi=20.0, p_neginf=0.1, p_nan=0.05, seed=N * 5 + D)
+    outputs, lses = wl.split_inputs(w)
+    ninf = float("-inf")
+    lses[:, 0, :] = ninf
+    lses[:-1, 1, :] = ninf
+    lses[-1, 1, :] = 7.5
+    lses[:, 2, 0] = torch.linspace(-80.0, 80.0, N)
+    outputs[N // 2, 3, 1] = float("nan")
+    lses[N // 2, 3, 1] = ninf
+    for base_e in (True, False):
+        y, g = _check(o, outputs, lses, base_e, f"wide rows N={N} D={D} {dtype} base_e={base_e}")
+        assert bool((y[0] == 0).all()) and bool((g[0] == -math.inf).all())
+        assert float(g[1, 0]) == 7.5 and torch.equal(y[1], outputs[-1, 1])
+        assert bool(torch.isnan(y[3, 1]).all())
