@@ -235,6 +235,22 @@ inline SplitShape varlen_shape(int N, int chunks, const SplitShape &plain) {
     return {G, cpl, cpl == 1 ? 8 : 4, true};
 }
 
+// The fused pack's per-row shape (rows that the 4-row group kernel does not take).  Its
+// packed-row stores favour more loads in flight per lane and no LSE prefetch: with 4-7
+// splits the variable-length shape (16 loads per lane), with 8 or more two slots of 8 splits,
+// both with the plain combine's lanes per row (so the result equals dcp_lse_combine +
+// dcp_pack bit for bit).  Measured at D = 512, B = 16384 (fractions of the measured peak, this
+// shape against the plain one): S = 4, 2-16 ranks: 0.97-0.98 against 0.85-0.89; S = 8:
+// 1.01 against 0.99; S = 16 (B = 4096): 1.03 against 1.00.
+inline SplitShape pack_shape(int N, int chunks, const SplitShape &plain) {
+    if (N >= 8 && plain.cpl == 2) return {plain.G, 2, 8, false};
+    if (N >= 4) {
+        const SplitShape v = varlen_shape(N, chunks, plain);
+        if (v.G == plain.G) return {v.G, v.cpl, v.nb, false};
+    }
+    return {plain.G, plain.cpl, plain.nb, false};
+}
+
 // Registers are capped so that 3 CTAs fit (8 loads in flight per lane), 4 for the 4-load
 // shape and 2 for the four-slot shapes, which spill otherwise.  Single-slot shapes only
 // arise with G = 4 or 8 and the 2 x 2 shape with G = 4 (rows of at most 8 chunks); a shape
@@ -248,6 +264,9 @@ int32_t launch_split_g(const dcp::CombineArgs &a, const SplitShape &s, cudaStrea
     }
     if constexpr (G <= 8) {
         if (s.cpl == 1) return launch_combine<T, G, 1, 8, false, 3, false, VARLEN, PACK_OUT, PREFETCH>(a, stream);
+    }
+    if constexpr (PACK_OUT) {
+        if (s.nb == 8) return launch_combine<T, G, 2, 8, false, 2, false, VARLEN, PACK_OUT, PREFETCH>(a, stream);
     }
     if constexpr (G == 4) {
         if (s.nb == 2) return launch_combine<T, 4, 2, 2, false, 4, false, VARLEN, PACK_OUT, PREFETCH>(a, stream);
@@ -287,8 +306,7 @@ int32_t dispatch_split(dcp::CombineArgs a, cudaStream_t stream) {
             a.red_lanes = s.G;  // the weights summed as the split combine would (same lanes per row)
             return dispatch_group_pack<T>(a, stream);
         }
-        if (s.prefetch) return launch_split<T, false, true, true>(a, s, stream);
-        return launch_split<T, false, true, false>(a, s, stream);
+        return launch_split<T, false, true, false>(a, pack_shape(a.N, a.chunks, s), stream);
     }
     if (s.prefetch) return launch_split<T, false, false, true>(a, s, stream);
     return launch_split<T, false, false, false>(a, s, stream);
