@@ -97,9 +97,9 @@ uint64_t magic64(uint64_t d) {
 // One pack kernel instance: its dynamic shared memory is reserved once per device (enough for
 // a stage of `max_stage_w` words), and its resident CTAs per SM are cached per device for the
 // last dynamic shared-memory size asked.
-template <int STAGES, int MAX_ROWS>
+template <int STAGES, int MAX_ROWS, bool RANK_FAST>
 struct PackInstance {
-    static constexpr auto kernel = dcp::pack_kernel<STAGES, dcp::kPackThreads, MAX_ROWS>;
+    static constexpr auto kernel = dcp::pack_kernel<STAGES, dcp::kPackThreads, MAX_ROWS, RANK_FAST>;
     static bool reserve(int max_stage_w) {
         static std::atomic<int> done[64];
         int dev = 0;
@@ -124,34 +124,44 @@ struct PackInstance {
     }
 };
 
-// Tile geometry and launch of one pack instance.  A stage holds about `stage_words` words of
+// Geometry of a pack instance for one call.  A stage holds about `stage_words` words of
 // source rows (at least one row, at most MAX_ROWS) and their LSE words, plus 4 words of slack
 // for the second aligned read of the last chunk.
-template <int STAGES, int MAX_ROWS>
-int32_t launch_pack(const char *fn, dcp::PackArgs a, int stage_words, bool runs_if_short, cudaStream_t stream) {
-    using I = PackInstance<STAGES, MAX_ROWS>;
-    a.tile_rows = (stage_words - 8) / a.row_pitch_w;
-    if (a.tile_rows < 1) a.tile_rows = 1;
-    if (a.tile_rows > MAX_ROWS) a.tile_rows = MAX_ROWS;
-    a.stage_w = ((a.tile_rows * a.row_pitch_w + 3) & ~3) + 4;
+struct PackGeom {
+    int tile_rows = 0;
+    int stage_w = 0;
+    size_t smem = 0;
+    int64_t tiles = 0;  // tiles of the call
+    int64_t cap = 0;    // CTAs resident at once
+};
+
+template <int STAGES, int MAX_ROWS, bool RANK_FAST = false>
+bool pack_geometry(const dcp::PackArgs &a, int stage_words, PackGeom &g) {
+    using I = PackInstance<STAGES, MAX_ROWS, RANK_FAST>;
+    g.tile_rows = (stage_words - 8) / a.row_pitch_w;
+    if (g.tile_rows < 1) g.tile_rows = 1;
+    if (g.tile_rows > MAX_ROWS) g.tile_rows = MAX_ROWS;
+    g.stage_w = ((g.tile_rows * a.row_pitch_w + 3) & ~3) + 4;
     const int max_stage_w = (int)(((kMaxD + 1 + 3) & ~int64_t(3)) + 4);  // one fp32 row of kMaxD words
-    if (!I::reserve(stage_words + 8 > max_stage_w ? stage_words + 8 : max_stage_w))
-        return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory for the pack kernel", fn);
-    const size_t smem = (size_t)STAGES * a.stage_w * 4;
-    const int per_sm = I::resident(smem);
-    const int64_t tiles = (a.rows + a.tile_rows - 1) / a.tile_rows;
-    const int64_t cap = (int64_t)sm_count() * per_sm;
-    // With contiguous heads, the rows of one (rank, token) can be copied as one run.  Measured
-    // on B200 (bf16, fraction of the measured copy peak): runs win for launches of at most
-    // ~24 tiles per CTA (N = 8, B = 1024, D = 512: 0.91 against 0.85; N = 2, B = 16384,
-    // D = 128: 0.88 against 0.80) and with rows of at most 128 bytes (D = 64: 0.84 against
-    // 0.57), and lose in longer launches of larger rows, where one copy per row keeps more
-    // copies in flight (N = 16, B = 16384: D = 512 0.94 against 0.87, D = 128 0.91 against 0.85).
+    if (!I::reserve(stage_words + 8 > max_stage_w ? stage_words + 8 : max_stage_w)) return false;
+    g.smem = (size_t)STAGES * g.stage_w * 4;
+    const int64_t per_rank = a.B * a.Hr;
+    g.tiles = RANK_FAST ? (a.rows / per_rank) * ((per_rank + g.tile_rows - 1) / g.tile_rows)
+                        : (a.rows + g.tile_rows - 1) / g.tile_rows;
+    g.cap = (int64_t)sm_count() * I::resident(g.smem);
+    return true;
+}
+
+// `runs`: where a token's heads are contiguous, the rows of one (rank, token) in a tile are
+// copied as one run.
+template <int STAGES, int MAX_ROWS, bool RANK_FAST = false>
+int32_t launch_pack(const char *fn, dcp::PackArgs a, const PackGeom &g, bool runs, cudaStream_t stream) {
+    a.tile_rows = g.tile_rows;
+    a.stage_w = g.stage_w;
     const bool contiguous = a.src_stride_h_w == a.data_w;
-    const bool runs = contiguous && (!runs_if_short || tiles <= 24 * cap);
-    a.max_run = runs ? (int32_t)(a.Hr < (int64_t(1) << 20) ? a.Hr : (int64_t(1) << 20)) : 1;
-    const int grid = (int)(tiles < cap ? tiles : cap);
-    I::kernel<<<grid, dcp::kPackThreads, smem, stream>>>(a);
+    a.max_run = runs && contiguous ? (int32_t)(a.Hr < (int64_t(1) << 20) ? a.Hr : (int64_t(1) << 20)) : 1;
+    const int grid = (int)(g.tiles < g.cap ? g.tiles : g.cap);
+    PackInstance<STAGES, MAX_ROWS, RANK_FAST>::kernel<<<grid, dcp::kPackThreads, g.smem, stream>>>(a);
     return launch_status(fn);
 }
 
@@ -462,12 +472,33 @@ int32_t pack_impl(const char *fn, const void *cp_attn_out, const float *cp_attn_
     a.wait_limit_ns = wait_limit_ns;
     a.stall_bytes = stall_bytes;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    // Rows of at most 128 bytes: 2 stages of up to 256 rows (about 32 KiB), copied as runs
-    // (D = 64: 0.84 of peak, against 0.72 for 3 stages of 64 rows with runs).  Otherwise 3
-    // stages of up to 64 rows or 32 KiB (measured best among 2-6 stages of 16-48 KiB and 64-256
-    // rows, which need the smaller stages' 4 CTAs per SM at D = 128).
-    if (a.data_w <= 32) return launch_pack<2, 256>(fn, a, 12288, false, stream);
-    return launch_pack<dcp::kPackStages, dcp::kPackMaxTileRows>(fn, a, dcp::kPackMinStageWords, true, stream);
+    // Shapes measured on B200 (bf16, fractions of the measured copy peak).
+    // * Rows of at most 128 bytes: 2 stages of up to 256 rows (about 32 KiB), copied as runs
+    //   (D = 64: 0.84, against 0.72 for 3 stages of 64 rows with runs and 0.57 without).
+    // * Otherwise 3 stages of up to 64 rows or 32 KiB (the best of 2-6 stages of 16-48 KiB and
+    //   64-256 rows; at D = 128 the 64-row tile keeps 4 CTAs on an SM).  Runs of a token's
+    //   contiguous heads win in launches of at most ~24 tiles per CTA (N = 8, B = 1024,
+    //   D = 512: 0.91 against 0.85; N = 2, B = 16384, D = 128: 0.88 against 0.80) and lose in
+    //   longer ones, where one copy per row keeps more copies in flight (N = 16, B = 16384:
+    //   D = 512 0.94 against 0.87, D = 128 0.91 against 0.85).
+    // * Longer launches of rows of 1 KiB and more for at most 4 ranks: 2 stages of up to 48 KiB,
+    //   tiles in rank-fastest order, so that the tiles in flight read all ranks of the same
+    //   tokens (D = 512: N = 2 0.97 against 0.95, N = 4 0.93 against 0.90; with 8 and 16 ranks
+    //   this order lost, 0.89-0.91 against 0.92-0.96).
+    PackGeom g;
+    if (a.data_w <= 32) {
+        if (!pack_geometry<2, 256>(a, 12288, g)) return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
+        return launch_pack<2, 256>(fn, a, g, true, stream);
+    }
+    if (!pack_geometry<dcp::kPackStages, dcp::kPackMaxTileRows>(a, dcp::kPackMinStageWords, g))
+        return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
+    if (g.tiles <= 24 * g.cap) return launch_pack<dcp::kPackStages, dcp::kPackMaxTileRows>(fn, a, g, true, stream);
+    if (a.data_w >= 256 && world_size <= 4) {
+        PackGeom r;
+        if (!pack_geometry<2, 256, true>(a, 12288, r)) return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
+        return launch_pack<2, 256, true>(fn, a, r, false, stream);
+    }
+    return launch_pack<dcp::kPackStages, dcp::kPackMaxTileRows>(fn, a, g, false, stream);
 }
 
 }  // namespace

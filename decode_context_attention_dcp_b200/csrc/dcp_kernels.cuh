@@ -1225,7 +1225,7 @@ __device__ __forceinline__ void pack_store_tile(const uint32_t *stage, uint32_t 
 //   the row's LSE word (rows are >= 5 words, so a chunk holds at most one LSE).
 //   The partial chunks at the two ends of the range use 4-byte stores.
 // Every word of the send buffer is written once, by one CTA.
-template <int STAGES = kPackStages, int THREADS = kPackThreads, int MAX_ROWS = kPackMaxTileRows>
+template <int STAGES = kPackStages, int THREADS = kPackThreads, int MAX_ROWS = kPackMaxTileRows, bool RANK_FAST = false>
 __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
     constexpr int kPackStages = STAGES;
     constexpr int kPackThreads = THREADS;
@@ -1238,7 +1238,12 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
     __shared__ uint64_t s_full[kPackStages];                      // a stage's rows have landed
     __shared__ int s_abort;                                       // a wait timed out
     const int tid = threadIdx.x;
-    const int64_t tiles = (a.rows + a.tile_rows - 1) / a.tile_rows;
+    // RANK_FAST: tiles never straddle a rank, and tile t is the (t / ranks)-th tile of rank
+    // t mod ranks, so the tiles in flight at once cover all ranks of the same tokens
+    const int64_t per_rank = a.B * a.Hr;
+    const int64_t ranks = a.rows / per_rank;
+    const int64_t tiles_per_rank = (per_rank + a.tile_rows - 1) / a.tile_rows;
+    const int64_t tiles = RANK_FAST ? ranks * tiles_per_rank : (a.rows + a.tile_rows - 1) / a.tile_rows;
     const int64_t my_tiles = tiles > blockIdx.x ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const int tile_rows = a.tile_rows;
     const int data_w = a.data_w;
@@ -1249,14 +1254,23 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
     const uint32_t *__restrict__ src = a.src;
     const uint32_t *__restrict__ lse = a.lse;
 
+    auto tile_start = [&](int64_t k) -> int64_t {  // the first packed row of this CTA's k-th tile
+        const int64_t t = blockIdx.x + k * gridDim.x;
+        if constexpr (RANK_FAST) {
+            const int64_t j = t / ranks;
+            return (t - j * ranks) * per_rank + j * tile_rows;
+        }
+        return t * tile_rows;
+    };
     auto tile_rows_of = [&](int64_t k) -> int {
-        const int64_t i0 = (blockIdx.x + k * gridDim.x) * tile_rows;
+        const int64_t i0 = tile_start(k);
+        if constexpr (RANK_FAST) return (int)min((int64_t)tile_rows, per_rank - i0 % per_rank);
         return (int)min((int64_t)tile_rows, a.rows - i0);
     };
     // row table of this CTA's k-th tile, into slot k % kPackStages: rows are
     // ordered [rank][token][head], row (rank, b, h) holds cp_attn_out[b, rank*Hr + h]
     auto fill_table = [&](int64_t k) {
-        const int64_t i0 = (blockIdx.x + k * gridDim.x) * tile_rows;
+        const int64_t i0 = tile_start(k);
         const int nrows = tile_rows_of(k);
         const int slot = (int)(k % kPackStages);
         for (int r = tid; r < nrows; r += kPackThreads) {
@@ -1338,7 +1352,7 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
             return;
         }
 
-        const int64_t i0 = (blockIdx.x + k * gridDim.x) * tile_rows;
+        const int64_t i0 = tile_start(k);
         pack_store_tile(s_stage + (int)(k % kPackStages) * stage_w, a.dst, i0 * pitch, tile_rows_of(k), data_w, pitch,
                         lse_base, pitch_magic, tid, kPackThreads);
         __syncthreads();  // stage k % kPackStages is free for tile k + kPackStages
