@@ -893,10 +893,16 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) online_unpack_kerne
             if (w != w) w = 0.0f;
             if (!mine) w = 0.0f;
             m = mn;
+            // the running sums are still +0 in the first batch, where scaling them changes nothing
+            if (n0 > 0) {
 #pragma unroll
-            for (int k = 0; k < CPL; ++k)
+                for (int k = 0; k < CPL; ++k)
 #pragma unroll
-                for (int e = 0; e < kE; ++e) acc[k][e] *= scale;
+                    for (int e = 0; e < kE; ++e) acc[k][e] *= scale;
+#pragma unroll
+                for (int e = 0; e < 3 * T::kPerWord; ++e) tacc[e] *= scale;
+                S *= scale;
+            }
             {
                 const uint32_t tw[3] = {t.w[0], t.w[1], t.w[2]};
 #pragma unroll
@@ -905,10 +911,9 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) online_unpack_kerne
                     T::decode(tw[e], f);
 #pragma unroll
                     for (int h = 0; h < T::kPerWord; ++h)
-                        tacc[e * T::kPerWord + h] = fmaf(w, f[h], tacc[e * T::kPerWord + h] * scale);
+                        tacc[e * T::kPerWord + h] = fmaf(w, f[h], tacc[e * T::kPerWord + h]);
                 }
             }
-            S *= scale;
 #pragma unroll
             for (int i = 0; i < NB; ++i) {
                 if (n0 + i >= a.N) break;  // the same for the whole warp
