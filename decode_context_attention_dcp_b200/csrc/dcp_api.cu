@@ -11,6 +11,7 @@
 
 #include <atomic>
 
+#include "dcp_combine_launch.cuh"
 #include "dcp_host.h"
 #include "dcp_testing.h"
 
@@ -510,6 +511,25 @@ int32_t dcp_pack(const void *cp_attn_out, const float *cp_attn_lse, void *send_b
                  void *cuda_stream) {
     return pack_impl("dcp_pack", cp_attn_out, cp_attn_lse, send_buf, B, H, D, world_size, dtype, out_stride_b,
                      out_stride_h, lse_stride_b, cuda_stream, dcp::kWaitLimitNs, 0u);
+}
+
+int32_t dcp_testing_split_shape(int32_t kind, int32_t N, int32_t chunks, int32_t *out) {
+    if (kind < 0 || kind > 2 || N < 1 || N > DCP_MAX_SHARDS || chunks < 1 || !out)
+        return fail(DCP_ERR_INVALID_ARG, "dcp_testing_split_shape: kind %d, N %d, chunks %d", (int)kind, (int)N,
+                    (int)chunks);
+    const dcp_host::SplitShape plain = dcp_host::split_shape(N, chunks);
+    dcp_host::SplitShape s = plain;
+    if (kind == 1) {
+        s = dcp_host::varlen_shape(N, chunks, plain);
+        if (dcp_host::varlen_all_in_flight(s, N, chunks)) s.nb = 8;
+    } else if (kind == 2) {
+        s = dcp_host::pack_shape(N, chunks, plain);
+    }
+    out[0] = s.G;
+    out[1] = s.cpl;
+    out[2] = s.nb;
+    out[3] = s.prefetch ? 1 : 0;
+    return ok();
 }
 
 int32_t dcp_testing_pack_stalled(const void *cp_attn_out, const float *cp_attn_lse, void *send_buf, int64_t B,

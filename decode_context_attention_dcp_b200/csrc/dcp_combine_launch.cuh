@@ -231,14 +231,22 @@ inline SplitShape split_shape(int N, int chunks) {
 //   D = 256, N = 4, 8, 16: 1.04, 1.04, 1.04 against 1.11, 1.09, 1.05
 //   D = 512, N = 4, 8, 16: 1.03, 1.05, 1.03 against 1.08, 1.08, 1.03
 inline SplitShape varlen_shape(int N, int chunks, const SplitShape &plain) {
-    if (N < 4) return plain;
+    const SplitShape kept = {plain.G, plain.cpl, plain.nb, true};  // the varlen kernel always prefetches
+    if (N < 4) return kept;
     int G = 4;
     while (G * 4 < chunks && G < 32) G *= 2;
     const int lo = G < plain.G ? G : plain.G;
-    if (G != plain.G && N > 2 * lo) return plain;
+    if (G != plain.G && N > 2 * lo) return kept;
     const int slots = (chunks + G - 1) / G;
     const int cpl = slots <= 2 ? slots : 4;
     return {G, cpl, cpl == 1 ? 8 : 4, true};
+}
+
+// The variable-length combine of 8 or more shards with 8 lanes per row of 144-256 bytes keeps
+// all 8 shards of a batch in flight: D = 128, B = 16384, N = 16 took 1.03 of the plain
+// combine's time per byte read, against 1.05 with 4.
+inline bool varlen_all_in_flight(const SplitShape &v, int N, int chunks) {
+    return v.G == 8 && v.cpl == 2 && chunks > 8 && chunks <= 16 && N >= 8;
 }
 
 // The fused pack's per-row shape (rows that the 4-row group kernel does not take).  Its
@@ -307,11 +315,8 @@ int32_t dispatch_split(dcp::CombineArgs a, cudaStream_t stream) {
     if (a.varlen) {
         const SplitShape v = varlen_shape(a.N, a.chunks, s);
         a.slots = (a.chunks + v.G - 1) / v.G;
-        if (v.G == 8 && v.cpl == 2 && a.chunks > 8 && a.chunks <= 16 && a.N >= 8) {
-            // all 8 shards of a batch in flight: D = 128, B = 16384, N = 16 took 1.03 of the
-            // plain combine's time per byte read, against 1.05 with 4
+        if (varlen_all_in_flight(v, a.N, a.chunks))
             return launch_combine<T, 8, 2, 8, false, 2, false, true, false, true>(a, stream);
-        }
         return launch_split<T, true, false, true>(a, v, stream);
     }
     if (a.pack_b > 0) {

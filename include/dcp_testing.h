@@ -1,7 +1,9 @@
 /*
- * dcp_testing.h -- test hook of libdcpcombine.so: makes the timeout path of the pack
+ * dcp_testing.h -- test hooks of libdcpcombine.so: one makes the timeout path of the pack
  * kernel's bounded wait run, so that a test can check it without faulting or hanging a
- * GPU.  Not part of the combine; no page has a counterpart.
+ * GPU; one reports the launch shape the host picks for a split-layout combine, so that the
+ * shape rules can be checked without a GPU.  Not part of the combine; no page has a
+ * counterpart.
  */
 #ifndef DCP_TESTING_H
 #define DCP_TESTING_H
@@ -24,6 +26,19 @@ int32_t dcp_testing_pack_stalled(const void *cp_attn_out, const float *cp_attn_l
                                  int64_t B, int64_t H, int64_t D, int32_t world_size, int32_t dtype,
                                  int64_t out_stride_b, int64_t out_stride_h, int64_t lse_stride_b,
                                  void *cuda_stream);
+
+/*
+ * The shape the host picks for a split-layout combine of N shards whose rows are `chunks`
+ * 16-byte chunks (D * elemsize / 16): kind 0 = dcp_lse_combine (and its strided form),
+ * 1 = dcp_lse_combine_varlen, 2 = the per-row path of dcp_combine_pack.  Writes out[0] =
+ * lanes per row, out[1] = chunk slots per lane per pass, out[2] = shards per batch, out[3] =
+ * 1 if phase 1's LSE reads are prefetched (for kind 0 before the short-launch rule, which
+ * also depends on the row count).  The lanes per row decide the result bits: the weights are
+ * summed by lane j of G over shards j, j + G, ..., then by halving over the G lanes.  Needs
+ * no GPU.  Returns DCP_OK, or DCP_ERR_INVALID_ARG for a kind outside 0..2, N outside
+ * [1, DCP_MAX_SHARDS], chunks < 1 or a null `out`.
+ */
+int32_t dcp_testing_split_shape(int32_t kind, int32_t N, int32_t chunks, int32_t *out);
 
 #ifdef __cplusplus
 }
