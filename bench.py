@@ -57,6 +57,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-chunks", type=int, default=8, help="token chunks pipelined over three streams")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -569,41 +570,69 @@ def run_ours(args) -> int:
                 "frac": dk["gbs"] / peak, "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json hbm_gbs' if peak_src == 'measured' else 'profiling recipe fallback'})",
                 "traffic": load_traffic(dom, w.name), "algorithmic_bytes_per_launch": dk["bytes_per_launch"]}
 
-    # end to end through the public API: pinned host inputs in, host result out, every step
+    # end to end through the public API: pinned host inputs in, host result out, every step.
+    # The step's tokens go in chunks over three streams (host-to-device copies, the two kernels,
+    # device-to-host copies), so that the copies in both directions and the kernels overlap,
+    # as a caller streaming a batch through the library would run it.
     e2e = None
     if not args.no_e2e:
         res_h = torch.empty(result.shape, dtype=result.dtype, pin_memory=True)
         glse_h = torch.empty(glse.shape, dtype=glse.dtype, pin_memory=True) if glse is not None else None
         d_out = torch.empty_like(cp_out)
         d_lse = torch.empty_like(cp_lse)
+        nc = max(1, min(args.e2e_chunks, w.B))
+        bounds = [(w.B * c // nc, w.B * (c + 1) // nc) for c in range(nc)]
+        sends = [torch.empty((w.N, b1 - b0, w.Hr, w.D + P), dtype=cp_out.dtype, device=device) for b0, b1 in bounds]
+        s_in, s_run, s_out = (torch.cuda.Stream(device=device) for _ in range(3))
+        ev = lambda: torch.cuda.Event()
+        in_done, run_done, out_done = [ev() for _ in bounds], [ev() for _ in bounds], [ev() for _ in bounds]
+        first = [True]
 
         def e2e_step():
-            d_out.copy_(cp_out_h, non_blocking=True)
-            d_lse.copy_(cp_lse_h, non_blocking=True)
-            dcp.dcp_pack(d_out, d_lse, send, w.N)
-            dcp.dcp_unpack_combine(send, result, glse, is_lse_base_on_e=w.is_lse_base_on_e,
-                                   return_lse=w.return_lse)
-            res_h.copy_(result, non_blocking=True)
-            if glse_h is not None:
-                glse_h.copy_(glse, non_blocking=True)
+            for c, (b0, b1) in enumerate(bounds):
+                with torch.cuda.stream(s_in):
+                    if not first[0]:
+                        s_in.wait_event(run_done[c])      # the last step's kernels have read this chunk
+                    d_out[b0:b1].copy_(cp_out_h[b0:b1], non_blocking=True)
+                    d_lse[b0:b1].copy_(cp_lse_h[b0:b1], non_blocking=True)
+                    in_done[c].record(s_in)
+                with torch.cuda.stream(s_run):
+                    s_run.wait_event(in_done[c])
+                    if not first[0]:
+                        s_run.wait_event(out_done[c])     # the last step's result chunk has left
+                    dcp.dcp_pack(d_out[b0:b1], d_lse[b0:b1], sends[c], w.N)
+                    dcp.dcp_unpack_combine(sends[c], result[b0:b1], None if glse is None else glse[b0:b1],
+                                           is_lse_base_on_e=w.is_lse_base_on_e, return_lse=w.return_lse)
+                    run_done[c].record(s_run)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(run_done[c])
+                    res_h[b0:b1].copy_(result[b0:b1], non_blocking=True)
+                    if glse_h is not None:
+                        glse_h[b0:b1].copy_(glse[b0:b1], non_blocking=True)
+                    out_done[c].record(s_out)
+            first[0] = False
 
-        with torch.cuda.stream(stream):
+        e2e_step()
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for st in (s_in, s_run, s_out):
+            st.wait_event(e0)
+        for _ in range(args.e2e_steps):
             e2e_step()
-            stream.synchronize()
-            barrier(device)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(args.e2e_steps):
-                e2e_step()
-            e1.record(stream)
+        for st in (s_in, s_run, s_out):
+            stream.wait_stream(st)
+        e1.record(stream)
         torch.cuda.synchronize(device)
         t_e2e = max_over_ranks(e0.elapsed_time(e1), device)
         h2d = cp_out.numel() * cp_out.element_size() + cp_lse.numel() * 4
         d2h = result.numel() * result.element_size() + (glse.numel() * 4 if glse is not None else 0)
         e2e = {"value": world * step_bytes * args.e2e_steps / (t_e2e * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-               "ms_per_step": t_e2e / args.e2e_steps}
-        del d_out, d_lse
+               "ms_per_step": t_e2e / args.e2e_steps, "token_chunks": nc,
+               "streams": "host-to-device copies, dcp_pack + dcp_unpack_combine, device-to-host copies"}
+        del d_out, d_lse, sends
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
