@@ -27,9 +27,9 @@ int32_t launch_combine(const dcp::CombineArgs &a, cudaStream_t stream) {
 }
 
 // The single-pass packed combine (online_unpack_kernel), one pass per row.
-template <class T, int G, int CPL, int NB, int MIN_CTAS>
-int32_t launch_online(const dcp::CombineArgs &a, cudaStream_t stream) {
-    auto kernel = dcp::online_unpack_kernel<T, G, CPL, NB, MIN_CTAS>;
+template <class T, int G, int CPL, int NB, int MIN_CTAS, bool SINGLE = false>
+int32_t launch_online_as(const dcp::CombineArgs &a, cudaStream_t stream) {
+    auto kernel = dcp::online_unpack_kernel<T, G, CPL, NB, MIN_CTAS, SINGLE>;
     static InstanceCache ic;
     if (a.slots > CPL) return fail(DCP_ERR_INVALID_ARG, "dcp_unpack_combine: internal shape error");
     constexpr int kUnitsPerWarp = 32 / G;
@@ -41,6 +41,13 @@ int32_t launch_online(const dcp::CombineArgs &a, cudaStream_t stream) {
     const int grid = (int)(want < cap ? want : cap);
     kernel<<<grid, dcp::kCombineThreads, 0, stream>>>(a);
     return launch_status("dcp_unpack_combine");
+}
+
+// ... with the single-batch instance when every shard fits one batch
+template <class T, int G, int CPL, int NB, int MIN_CTAS>
+int32_t launch_online(const dcp::CombineArgs &a, cudaStream_t stream) {
+    if (a.N <= NB) return launch_online_as<T, G, CPL, NB, MIN_CTAS, true>(a, stream);
+    return launch_online_as<T, G, CPL, NB, MIN_CTAS, false>(a, stream);
 }
 
 // Occupancy: the kernel keeps NB * CPL 16-byte loads in flight per lane, so the
@@ -161,7 +168,7 @@ int32_t dispatch_packed(dcp::CombineArgs a, cudaStream_t stream) {
         if (chunks <= 16) {
             if (a.N >= 8) {
                 a.slots = (chunks + 7) / 8;
-                return launch_online<T, 8, 2, 4, 3>(a, stream);
+                return launch_online_as<T, 8, 2, 4, 3>(a, stream);
             }
             a.slots = (chunks + 3) / 4;
             return launch_online<T, 4, 4, 4, 2>(a, stream);

@@ -817,7 +817,10 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) combine_kernel(cons
 // weights formed against the running maximum and rescaled to the final one, so it differs from
 // the two-phase result by fp32 rounding only.  Row layout, realignment and stores are those of
 // combine_kernel's uniform packed path (G lanes per row, CPL chunk slots per lane).
-template <class T, int G, int CPL, int NB, int MIN_CTAS>
+// SINGLE (N <= NB, so one batch holds every shard): the batch's maximum is the row's, its weight
+// sum is the row's S, and the weights are normalised before the weighted sum, in the page's
+// order, instead of rescaling the sums at the end.
+template <class T, int G, int CPL, int NB, int MIN_CTAS, bool SINGLE = false>
 __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) online_unpack_kernel(const CombineArgs a) {
     static_assert(NB <= G, "each shard of a batch needs a lane to read its tail chunk");
     constexpr int kUnitsPerWarp = 32 / G;
@@ -879,62 +882,95 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) online_unpack_kerne
         float tacc[3 * T::kPerWord];  // this lane's shards: weighted sum of the tail chunks' first 3 words
 #pragma unroll
         for (int e = 0; e < 3 * T::kPerWord; ++e) tacc[e] = 0.0f;
-
-        for (int n0 = 0; n0 < a.N; n0 += NB) {
-            if (n0 > 0) issue(n0);
-            // the batch's LSEs, its maximum and the rescaling of the running state
-            const bool mine = valid && j < NB && n0 + j < a.N;
-            const uint32_t lbits = q == 0 ? t.w[0] : q == 1 ? t.w[1] : q == 2 ? t.w[2] : t.w[3];
-            const float l = mine ? sanitize_lse(lbits) : -INFINITY;
-            const float bmax = group_max<G>(l);
-            const float mn = fmaxf(m, bmax);
-            const float scale = mn == -INFINITY ? 1.0f : (base_e ? expf(m - mn) : exp2f(m - mn));
-            float w = base_e ? expf(l - mn) : exp2f(l - mn);
-            if (w != w) w = 0.0f;
-            if (!mine) w = 0.0f;
-            m = mn;
-            // the running sums are still +0 in the first batch, where scaling them changes nothing
-            if (n0 > 0) {
+        // the tail chunk's first 3 words, weighted into tacc
+        auto add_tail = [&](float w) {
+            const uint32_t tw[3] = {t.w[0], t.w[1], t.w[2]};
 #pragma unroll
-                for (int k = 0; k < CPL; ++k)
+            for (int e = 0; e < 3; ++e) {
+                float f[T::kPerWord];
+                T::decode(tw[e], f);
 #pragma unroll
-                    for (int e = 0; e < kE; ++e) acc[k][e] *= scale;
-#pragma unroll
-                for (int e = 0; e < 3 * T::kPerWord; ++e) tacc[e] *= scale;
-                S *= scale;
+                for (int h = 0; h < T::kPerWord; ++h)
+                    tacc[e * T::kPerWord + h] = fmaf(w, f[h], tacc[e * T::kPerWord + h]);
             }
-            {
-                const uint32_t tw[3] = {t.w[0], t.w[1], t.w[2]};
+        };
+        auto add_rows = [&](int i, float wi) {
 #pragma unroll
-                for (int e = 0; e < 3; ++e) {
+            for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
                     float f[T::kPerWord];
-                    T::decode(tw[e], f);
+                    T::decode(x[i][k].w[e], f);
 #pragma unroll
                     for (int h = 0; h < T::kPerWord; ++h)
-                        tacc[e * T::kPerWord + h] = fmaf(w, f[h], tacc[e * T::kPerWord + h]);
+                        acc[k][e * T::kPerWord + h] = fmaf(wi, f[h], acc[k][e * T::kPerWord + h]);
                 }
-            }
+        };
+        float r = 1.0f;  // the normalisation still to apply to the sums (1: already in the weights)
+        if constexpr (SINGLE) {
+            const bool mine = valid && j < a.N;
+            const uint32_t lbits = q == 0 ? t.w[0] : q == 1 ? t.w[1] : q == 2 ? t.w[2] : t.w[3];
+            const float l = mine ? sanitize_lse(lbits) : -INFINITY;
+            m = group_max<G>(l);
+            float w = base_e ? expf(l - m) : exp2f(l - m);
+            if (w != w) w = 0.0f;
+            if (!mine) w = 0.0f;
+            float wv[NB];
 #pragma unroll
             for (int i = 0; i < NB; ++i) {
-                if (n0 + i >= a.N) break;  // the same for the whole warp
-                const float wi = __shfl_sync(0xffffffffu, w, row_lane0 + i);
-                S += wi;
-#pragma unroll
-                for (int k = 0; k < CPL; ++k)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float f[T::kPerWord];
-                        T::decode(x[i][k].w[e], f);
-#pragma unroll
-                        for (int h = 0; h < T::kPerWord; ++h)
-                            acc[k][e * T::kPerWord + h] = fmaf(wi, f[h], acc[k][e * T::kPerWord + h]);
-                    }
+                wv[i] = 0.0f;
+                if (i >= a.N) break;  // the same for the whole warp
+                wv[i] = __shfl_sync(0xffffffffu, w, row_lane0 + i);
+                S += wv[i];
             }
-        }
-        // normalise by the clamped sum; the tail sums over the row's lanes
-        const float r = 1.0f / fmaxf(S, 1e-10f);
+            const float rn = 1.0f / fmaxf(S, 1e-10f);
+            add_tail(w * rn);
 #pragma unroll
-        for (int e = 0; e < 3 * T::kPerWord; ++e) tacc[e] = group_sum<G>(tacc[e]) * r;
+            for (int i = 0; i < NB; ++i) {
+                if (i >= a.N) break;  // the same for the whole warp
+                add_rows(i, wv[i] * rn);
+            }
+        } else {
+            for (int n0 = 0; n0 < a.N; n0 += NB) {
+                if (n0 > 0) issue(n0);
+                // the batch's LSEs, its maximum and the rescaling of the running state
+                const bool mine = valid && j < NB && n0 + j < a.N;
+                const uint32_t lbits = q == 0 ? t.w[0] : q == 1 ? t.w[1] : q == 2 ? t.w[2] : t.w[3];
+                const float l = mine ? sanitize_lse(lbits) : -INFINITY;
+                const float bmax = group_max<G>(l);
+                const float mn = fmaxf(m, bmax);
+                const float scale = mn == -INFINITY ? 1.0f : (base_e ? expf(m - mn) : exp2f(m - mn));
+                float w = base_e ? expf(l - mn) : exp2f(l - mn);
+                if (w != w) w = 0.0f;
+                if (!mine) w = 0.0f;
+                m = mn;
+                // the running sums are still +0 in the first batch, where scaling them changes nothing
+                if (n0 > 0) {
+#pragma unroll
+                    for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                        for (int e = 0; e < kE; ++e) acc[k][e] *= scale;
+#pragma unroll
+                    for (int e = 0; e < 3 * T::kPerWord; ++e) tacc[e] *= scale;
+                    S *= scale;
+                }
+                add_tail(w);
+#pragma unroll
+                for (int i = 0; i < NB; ++i) {
+                    if (n0 + i >= a.N) break;  // the same for the whole warp
+                    const float wi = __shfl_sync(0xffffffffu, w, row_lane0 + i);
+                    S += wi;
+                    add_rows(i, wi);
+                }
+            }
+            r = 1.0f / fmaxf(S, 1e-10f);
+        }
+        // the tail sums over the row's lanes, normalised
+#pragma unroll
+        for (int e = 0; e < 3 * T::kPerWord; ++e) {
+            tacc[e] = group_sum<G>(tacc[e]);
+            if constexpr (!SINGLE) tacc[e] *= r;
+        }
         if (a.return_lse && valid && j == 0) a.glse[u] = (base_e ? logf(S) : log2f(S)) + (m == -INFINITY ? 0.0f : m);
         // round, then realign: result chunk c = words q.. of sums c and c + 1 (the next lane's, lane
         // 0's next slot for lane G - 1, the tail sums for the row's last chunk)
@@ -945,7 +981,7 @@ __global__ void __launch_bounds__(kCombineThreads, MIN_CTAS) online_unpack_kerne
             for (int e = 0; e < 4; ++e) {
                 float f[T::kPerWord];
 #pragma unroll
-                for (int h = 0; h < T::kPerWord; ++h) f[h] = acc[k][e * T::kPerWord + h] * r;
+                for (int h = 0; h < T::kPerWord; ++h) f[h] = SINGLE ? acc[k][e * T::kPerWord + h] : acc[k][e * T::kPerWord + h] * r;
                 enc[k].w[e] = T::encode(f);
             }
         Words<4> tenc;
