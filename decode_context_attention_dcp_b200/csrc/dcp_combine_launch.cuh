@@ -149,9 +149,14 @@ int32_t dispatch_packed(dcp::CombineArgs a, cudaStream_t stream) {
     // (two shards, or packed rows of 1 KiB and more), and 2-4% slower where the stream
     // already hides it.
     const bool prefetch = a.N <= 2 || chunks >= 64;
-    if (uniform && a.N == 2 && chunks > 8 && chunks <= 16) {
-        // two shards, rows of 144-256 bytes: the single-pass kernel with both shards in one
-        // batch (B = 16384, D = 128: 0.80 of the measured peak against 0.76 two-phase)
+    if (uniform && a.N == 2 && chunks <= 16) {
+        // two shards, rows of at most 256 bytes: the single-pass kernel with both shards in one
+        // batch (B = 16384, D = 128: 0.84 of the measured peak against 0.76 two-phase; D = 64:
+        // 0.64 against 0.51)
+        if (chunks <= 8) {
+            a.slots = (chunks + 3) / 4;
+            return launch_online<T, 4, 2, 4, 3>(a, stream);
+        }
         a.slots = (chunks + 3) / 4;
         return launch_online<T, 4, 4, 2, 2>(a, stream);
     }
