@@ -182,6 +182,15 @@ int32_t dispatch_packed(dcp::CombineArgs a, cudaStream_t stream) {
         return launch_online<T, 8, 4, 4, 2>(a, stream);
     }
     if (uniform) {
+        if (chunks > 32 && chunks <= 64 && a.N <= 4) {
+            // rows of 513 bytes to 1 KiB and at most 4 shards: the single-pass kernel, one batch
+            // holding every shard (16 lanes per row).  Measured at D = 512 (fractions of the
+            // measured peak, against the two-phase kernel): B = 16384, N = 2, 3, 4: 0.92, 0.99,
+            // 0.97 against 0.885, 0.94, 0.95; B = 4096, N = 2, 4: 0.84, 1.00 against 0.79, 0.965.
+            a.slots = (chunks + 15) / 16;
+            if (a.N <= 2) return launch_online_as<T, 16, 4, 2, 2, true>(a, stream);
+            return launch_online_as<T, 16, 4, 4, 2, true>(a, stream);
+        }
         if (chunks > 32 && chunks <= 64 && a.N >= 3 && a.N < 16) {
             // rows of 513 bytes to 1 KiB and 3-15 shards: 16 lanes per row (a quarter of the
             // row's chunks per lane), 4 shards per batch (16 loads in flight per lane).

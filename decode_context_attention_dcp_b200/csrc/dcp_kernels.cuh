@@ -285,7 +285,8 @@ struct CombineArgs {
 // n * interleave < seq); a token outside every request has none.
 __device__ __forceinline__ int varlen_held_shards(const CombineArgs &a, int32_t seq) {
     if (seq <= 0) return 0;
-    const int32_t k = (seq - 1) / a.interleave + 1;
+    // interleave 1 (token-by-token sharding, the default) needs no division
+    const int32_t k = a.interleave == 1 ? seq : (seq - 1) / a.interleave + 1;
     return k < a.N ? k : a.N;
 }
 

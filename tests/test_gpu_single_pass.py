@@ -92,10 +92,11 @@ def test_full_size_single_pass(o):
 
 
 @pytest.mark.parametrize("dtype,D", [("bf16", 512), ("fp16", 512), ("fp32", 256), ("bf16", 264), ("bf16", 320)])
-@pytest.mark.parametrize("N", [3, 4, 5, 8, 15, 16])
+@pytest.mark.parametrize("N", [1, 2, 3, 4, 5, 8, 15, 16])
 def test_wide_rows_quarter_lanes(o, dtype, D, N):
-    """Packed rows of 513 bytes to 1 KiB with 3-15 shards take the two-phase kernel with 16
-    lanes per row (16 shards: 32 lanes); the same special rows as above, against the oracle.
+    """Packed rows of 513 bytes to 1 KiB: with 2-4 shards the single-pass kernel with one batch
+    and 16 lanes per row, with 5-15 the two-phase kernel with 16 lanes, with 16 (and 1) the
+    32-lane two-phase shape; the same special rows as above, against the oracle.
     12 tokens of 3 heads keep every shard's stride a multiple of 16 bytes."""
     B, Hr = 12, 3
     w = wl.CombineWorkload(f"wide_N{N}_D{D}_{dtype}", N=N, B=B, Hr=Hr, D=D, dtype=dtype, lse_lo=-20.0,
