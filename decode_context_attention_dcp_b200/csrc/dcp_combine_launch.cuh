@@ -73,25 +73,21 @@ int32_t launch_g(dcp::CombineArgs a, int G, int cpl, cudaStream_t stream) {
     }
 }
 
-// Shape of the work per lane.  Each lane should keep about eight 16-byte loads
-// in flight: chunk slots per lane (CPL) times shards per batch (NB = 8 / CPL),
-// so fewer shards ask for more chunks per lane, i.e. fewer lanes per row (G).
-// When all shards of the packed buffer put a row at the same offset from a
-// 16-byte boundary (the shard stride is a multiple of 16 bytes) and one pass
-// covers a row, the sums are realigned once per output chunk ("uniform");
-// otherwise every shard's chunk is realigned, and that path keeps at least two
-// slots per lane.
+// Shape of the packed two-phase combine.  Each lane should keep about eight 16-byte loads
+// in flight: chunk slots per lane (CPL) times shards per batch (NB = 8 / CPL), so fewer
+// shards ask for more chunks per lane, i.e. fewer lanes per row (G).  When all shards of the
+// packed buffer put a row at the same offset from a 16-byte boundary (the shard stride is a
+// multiple of 16 bytes) and one pass covers a row, the sums are realigned once per output
+// chunk ("uniform"); otherwise every shard's chunk is realigned, and that path keeps at least
+// two slots per lane.
 struct CombineShape {
     int G;    // lanes per row
     int cpl;  // chunk slots per lane per pass
 };
 
-inline CombineShape combine_shape(bool packed, bool uniform, int N, int chunks) {
+inline CombineShape combine_shape(bool uniform, int N, int chunks) {
     int cpl_target = N >= 8 ? 1 : N >= 4 ? 2 : 4;
-    if (packed && !uniform && cpl_target < 2) cpl_target = 2;
-    // split layout, 8 or more shards, rows of at most 256 bytes: two chunk slots per lane
-    // (four rows per warp) measured 3-6% faster than one with 8-15 shards, 2% with 16
-    if (!packed && N >= 8 && chunks <= 16) cpl_target = 2;
+    if (!uniform && cpl_target < 2) cpl_target = 2;
     const int per_lane = (chunks + cpl_target - 1) / cpl_target;
     int G = 4;
     while (G < per_lane && G < 32) G *= 2;
@@ -142,7 +138,7 @@ template <class T>
 int32_t dispatch_packed(dcp::CombineArgs a, cudaStream_t stream) {
     const int chunks = a.chunks;
     const bool uniform = (a.N == 1 || a.shard_stride_w % 4 == 0) && chunks <= 4 * 32;
-    const CombineShape sh = combine_shape(true, uniform, a.N, chunks);
+    const CombineShape sh = combine_shape(uniform, a.N, chunks);
     const int G = sh.G, cpl = sh.cpl;
     a.slots = (chunks + G - 1) / G;
     // Phase 1's reads one task ahead: measured worth it where phase 1's latency is exposed
@@ -162,10 +158,11 @@ int32_t dispatch_packed(dcp::CombineArgs a, cudaStream_t stream) {
     }
     if (uniform && chunks <= 32 && a.N >= 3) {
         // rows of at most 512 bytes and 3 or more shards: the single-pass kernel, whose LSEs
-        // come with each batch's data.  Measured at B = 16384 (fractions of the measured
-        // peak, single-pass against two-phase): D = 64 N = 8, 16: 0.91, 0.99 vs 0.74, 0.77;
-        // D = 128 N = 3, 4, 8, 16: 0.86, 0.96, 0.99, 1.03 vs 0.71, 0.77, 0.94, 0.91;
-        // D = 256 N = 4, 8: 0.96, 0.98 vs 0.82, 0.81.  At N = 2 the two kinds tie.
+        // come with each batch's data (with N <= 4 one batch holds them all).  Measured at
+        // B = 16384 (fractions of the measured peak, single-pass against two-phase): D = 64
+        // N = 4, 8, 16: 0.85, 0.91, 0.99 vs -, 0.74, 0.77; D = 128 N = 3, 4, 8, 16: 0.92,
+        // 0.97, 1.01, 1.03 vs 0.71, 0.77, 0.94, 0.91; D = 256 N = 3, 4, 8: 0.96, 0.99, 0.95
+        // vs -, 0.82, 0.81.
         if (chunks <= 8) {
             a.slots = (chunks + 3) / 4;
             return launch_online<T, 4, 2, 4, 3>(a, stream);
@@ -191,14 +188,14 @@ int32_t dispatch_packed(dcp::CombineArgs a, cudaStream_t stream) {
             if (a.N <= 2) return launch_online_as<T, 16, 4, 2, 2, true>(a, stream);
             return launch_online_as<T, 16, 4, 4, 2, true>(a, stream);
         }
-        if (chunks > 32 && chunks <= 64 && a.N >= 3 && a.N < 16) {
-            // rows of 513 bytes to 1 KiB and 3-15 shards: 16 lanes per row (a quarter of the
+        if (chunks > 32 && chunks <= 64 && a.N >= 5 && a.N < 16) {
+            // rows of 513 bytes to 1 KiB and 5-15 shards: 16 lanes per row (a quarter of the
             // row's chunks per lane), 4 shards per batch (16 loads in flight per lane).
-            // Measured at D = 512 (fractions of the measured peak, against the previous shape:
-            // 32 lanes per row, or 2 shards per batch at N = 3): B = 16384, N = 3, 4, 6, 8:
-            // 0.93, 0.94, 0.96, 0.96 against 0.87, 0.90, 0.92, 0.93; B = 4096, N = 4, 8: 1.00,
-            // 1.03 against 0.81, 1.00; B = 1024, N = 8: 0.81 against 0.81.  With 16 shards the
-            // 32-lane shape stays ahead (B = 4096: 1.03 against 0.98).
+            // Measured at D = 512 (fractions of the measured peak, against 32 lanes per row):
+            // B = 16384, N = 6, 8: 0.96, 0.96 against 0.92, 0.93; B = 4096, N = 8: 1.03 against
+            // 1.00; B = 1024, N = 8: 0.81 against 0.81.  The single-pass kernel (8 shards per
+            // batch) did not beat it at N = 5-8.  With 16 shards the 32-lane shape stays ahead
+            // (B = 4096: 1.03 against 0.98).
             a.slots = (chunks + 15) / 16;
             return launch_combine<T, 16, 4, 4, true, 2, true, false, false, true>(a, stream);
         }

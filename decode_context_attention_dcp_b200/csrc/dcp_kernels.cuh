@@ -6,9 +6,12 @@
 //   combine_kernel<..., PACKED=false>  combine of split receive buffers (any strides)
 //     VARLEN=true                      ... per request: shards without KV are not read
 //     PACK_OUT=true                    ... written as packed send rows (split merge + pack)
-//   combine_kernel<..., PACKED=true>   fused unpack + combine of the packed buffer
+//   combine_kernel<..., PACKED=true>   fused unpack + combine of the packed buffer (two phases)
 //     PREFETCH=true (either layout)    phase 1's reads copied one task ahead
-//   pack_kernel                         output rows + fp32 LSE -> packed rows (bulk copies)
+//   online_unpack_kernel               the same in one pass, LSEs arriving with each batch's
+//                                      data (packed rows of at most 1 KiB)
+//   group_pack_kernel                  split merge written as 4-row spans of packed send rows
+//   pack_kernel                        output rows + fp32 LSE -> packed rows (bulk copies)
 //
 // The combine follows vLLM API docs, vllm.v1.attention.ops.dcp_alltoall,
 // _lse_weighted_combine; the packed layout [N, B, H/N, D + P] follows the same
