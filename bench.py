@@ -63,7 +63,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the JSON line: per-kernel GB/s on every workload, as a markdown table")
-    ap.add_argument("--sweep-reps", type=int, default=20)
+    ap.add_argument("--sweep-reps", type=int, default=50)
     ap.add_argument("--points", default="",
                     help="--sweep: comma-separated workload names to run (default: every workload)")
     ap.add_argument("--kernels", default="",
