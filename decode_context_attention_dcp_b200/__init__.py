@@ -71,6 +71,8 @@ def library() -> ctypes.CDLL:
                 lib.dcp_pack.restype = _i32
                 lib.dcp_testing_pack_stalled.argtypes = lib.dcp_pack.argtypes
                 lib.dcp_testing_pack_stalled.restype = _i32
+                lib.dcp_testing_last_pack_kernel.argtypes = []
+                lib.dcp_testing_last_pack_kernel.restype = _i32
                 lib.dcp_lse_combine.argtypes = [_ptr, _ptr, _ptr, _ptr, _i32, _i64, _i64, _i64, _i64, _i64, _i32,
                                                 _i32, _i32, _ptr]
                 lib.dcp_lse_combine.restype = _i32

@@ -4,6 +4,8 @@
 // Host side only: argument validation (before any CUDA call), choice of the
 // kernel instance for the row width, grid sizing, launch, and launch-error
 // reporting.  Nothing here allocates device memory or synchronises.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdarg.h>
 #include <stdint.h>
@@ -95,6 +97,9 @@ uint64_t magic64(uint64_t d) {
 
 // The pack kernel's dynamic shared memory can exceed the default 48 KiB: opt in
 // once per device, for the largest stage any accepted row width needs.
+// The pack kernel this host thread launched last (dcp_testing_last_pack_kernel).
+thread_local int32_t t_last_pack_kernel = 0;
+
 // One pack kernel instance: its dynamic shared memory is reserved once per device (enough for
 // a stage of `max_stage_w` words), and its resident CTAs per SM are cached per device for the
 // last dynamic shared-memory size asked.
@@ -163,6 +168,117 @@ int32_t launch_pack(const char *fn, dcp::PackArgs a, const PackGeom &g, bool run
     a.max_run = runs && contiguous ? (int32_t)(a.Hr < (int64_t(1) << 20) ? a.Hr : (int64_t(1) << 20)) : 1;
     const int grid = (int)(g.tiles < g.cap ? g.tiles : g.cap);
     PackInstance<STAGES, MAX_ROWS, RANK_FAST>::kernel<<<grid, dcp::kPackThreads, g.smem, stream>>>(a);
+    t_last_pack_kernel = RANK_FAST ? 3 : a.max_run > 1 ? 2 : 1;
+    return launch_status(fn);
+}
+
+// ---- the tensor-copy pack (pack_tma_kernel) ----
+
+// cuTensorMapEncodeTiled, found once through the runtime (the library does not link the driver).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+    static std::atomic<int> tried{0};
+    PFN_cuTensorMapEncodeTiled_v12000 f = fn.load(std::memory_order_acquire);
+    if (f || tried.load(std::memory_order_acquire)) return f;
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    fn.store(f, std::memory_order_release);
+    tried.store(1, std::memory_order_release);
+    return f;
+}
+
+constexpr int kPackTmaStages = 2;
+constexpr int kPackTmaBoxBytes = 65536;  // about 64 KiB of rows per tile
+// the largest stage: 64 KiB of rows of at least 16 bytes (4096 rows), their LSE words, slack
+constexpr int kPackTmaMaxStageW = ((kPackTmaBoxBytes / 4 + kPackTmaBoxBytes / 16 + 4) + 31) & ~31;
+
+// A tensor map and tile shape for pack_tma_kernel, or false when the shape does not suit it
+// (more than 256 heads per rank, a token's heads over 64 KiB, no row split into pieces of at
+// most 256 elements and a multiple of 16 bytes, or an encoding the driver refuses).
+bool pack_tma_plan(dcp::PackArgs &a, const void *cp_attn_out, int64_t H, int64_t D, int es, int64_t out_stride_b,
+                   int64_t out_stride_h, CUtensorMap &map, int &dims) {
+    const int64_t row_bytes = (int64_t)a.data_w * 4;
+    if (a.Hr > 256 || a.Hr * row_bytes > kPackTmaBoxBytes) return false;
+    int64_t k = kPackTmaBoxBytes / (a.Hr * row_bytes);
+    if (k > 256) k = 256;
+    if (k > a.B) k = a.B;
+    int64_t m = (D + 255) / 256;  // pieces per row
+    while (m <= 256 && (D % m != 0 || ((D / m) * es) % 16 != 0)) ++m;
+    if (m > 256) return false;
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (!encode) return false;
+    const CUtensorMapDataType type = es == 4 ? CU_TENSOR_MAP_DATA_TYPE_UINT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+    const cuuint32_t one[4] = {1, 1, 1, 1};
+    CUresult r;
+    if (m == 1) {
+        const cuuint64_t dim[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)a.B};
+        const cuuint64_t stride[2] = {(cuuint64_t)(out_stride_h * es), (cuuint64_t)(out_stride_b * es)};
+        const cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)a.Hr, (cuuint32_t)k};
+        r = encode(&map, type, 3, const_cast<void *>(cp_attn_out), dim, stride, box, one, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        dims = 3;
+    } else {
+        const cuuint64_t dim[4] = {(cuuint64_t)(D / m), (cuuint64_t)m, (cuuint64_t)H, (cuuint64_t)a.B};
+        const cuuint64_t stride[3] = {(cuuint64_t)((D / m) * es), (cuuint64_t)(out_stride_h * es),
+                                      (cuuint64_t)(out_stride_b * es)};
+        const cuuint32_t box[4] = {(cuuint32_t)(D / m), (cuuint32_t)m, (cuuint32_t)a.Hr, (cuuint32_t)k};
+        r = encode(&map, type, 4, const_cast<void *>(cp_attn_out), dim, stride, box, one, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        dims = 4;
+    }
+    if (r != CUDA_SUCCESS) return false;
+    a.tile_tokens = (int32_t)k;
+    const int box_rows = (int)(k * a.Hr);
+    a.stage_w = ((box_rows * a.data_w + box_rows + 4) + 31) & ~31;  // 128-byte aligned stages
+    return true;
+}
+
+template <int DIMS>
+int32_t launch_pack_tma(const char *fn, const dcp::PackArgs &a, const CUtensorMap &map, cudaStream_t stream) {
+    auto kernel = dcp::pack_tma_kernel<kPackTmaStages, dcp::kPackThreads, DIMS, false>;
+    auto tail_kernel = dcp::pack_tma_kernel<kPackTmaStages, dcp::kPackThreads, DIMS, true>;
+    static std::atomic<int> reserved[64];
+    static std::atomic<uint64_t> occupancy[64];  // per device: (smem << 16) | ctas
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(DCP_ERR_CUDA, "%s: no device", fn);
+    if (!reserved[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kPackTmaStages * kPackTmaMaxStageW * 4 + 128) != cudaSuccess ||
+            cudaFuncSetAttribute(tail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kPackTmaStages * kPackTmaMaxStageW * 4 + 128) != cudaSuccess)
+            return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory for the pack kernel", fn);
+        reserved[dev].store(1, std::memory_order_release);
+    }
+    const size_t smem = (size_t)kPackTmaStages * a.stage_w * 4 + 128;  // + room to align the stages
+    int per_sm;
+    const uint64_t c = occupancy[dev].load(std::memory_order_relaxed);
+    if (c && (c >> 16) == smem) {
+        per_sm = (int)(c & 0xffff);
+    } else {
+        per_sm = resident_ctas(kernel, dcp::kPackThreads, smem);
+        occupancy[dev].store(((uint64_t)smem << 16) | (uint64_t)per_sm, std::memory_order_relaxed);
+    }
+    // whole tiles of tile_tokens tokens (B >= tile_tokens), then one tile per rank for the
+    // B mod tile_tokens tokens left
+    const int64_t ranks = a.rows / (a.B * a.Hr);
+    const int64_t cap = (int64_t)sm_count() * per_sm;
+    dcp::PackArgs m = a;
+    m.store_tokens = a.tile_tokens;
+    m.tiles_per_rank = a.B / a.tile_tokens;
+    m.first_token = 0;
+    const int64_t tiles = ranks * m.tiles_per_rank;
+    kernel<<<(int)(tiles < cap ? tiles : cap), dcp::kPackThreads, smem, stream>>>(map, m);
+    const int64_t rem = a.B % a.tile_tokens;
+    if (rem) {
+        m.store_tokens = (int32_t)rem;
+        m.tiles_per_rank = 1;
+        m.first_token = a.B - rem;
+        tail_kernel<<<(int)(ranks < cap ? ranks : cap), dcp::kPackThreads, smem, stream>>>(map, m);
+    }
+    t_last_pack_kernel = DIMS == 3 ? 4 : 5;
     return launch_status(fn);
 }
 
@@ -433,6 +549,7 @@ namespace {
 int32_t pack_impl(const char *fn, const void *cp_attn_out, const float *cp_attn_lse, void *send_buf, int64_t B,
                   int64_t H, int64_t D, int32_t world_size, int32_t dtype, int64_t out_stride_b, int64_t out_stride_h,
                   int64_t lse_stride_b, void *cuda_stream, uint64_t wait_limit_ns, uint32_t stall_bytes) {
+    t_last_pack_kernel = 0;
     int32_t st = check_common(fn, dtype, world_size, B, H, D);
     if (st != DCP_OK) return st;
     if (H % world_size != 0)
@@ -482,18 +599,31 @@ int32_t pack_impl(const char *fn, const void *cp_attn_out, const float *cp_attn_
     //   D = 512: 0.91 against 0.85; N = 2, B = 16384, D = 128: 0.88 against 0.80) and lose in
     //   longer ones, where one copy per row keeps more copies in flight (N = 16, B = 16384:
     //   D = 512 0.94 against 0.87, D = 128 0.91 against 0.85).
-    // * Longer launches of rows of 1 KiB and more for at most 4 ranks: 2 stages of up to 48 KiB,
+    // * Longer launches of rows of 1 KiB and more for 3 or 4 ranks: 2 stages of up to 48 KiB,
     //   tiles in rank-fastest order, so that the tiles in flight read all ranks of the same
-    //   tokens (D = 512: N = 2 0.97 against 0.95, N = 4 0.93 against 0.90; with 8 and 16 ranks
-    //   this order lost, 0.89-0.91 against 0.92-0.96).
+    //   tokens (D = 512, N = 4: 0.94 against 0.93 for the tensor copies below and 0.90 in rank
+    //   order; with 8 and 16 ranks this order lost, 0.89-0.91 against 0.92-0.96).
+    // * Longer launches otherwise: one tensor copy per tile of about 64 KiB (tokens x all heads of a
+    //   rank), 2 stages, one CTA per SM: D = 512, N = 8 / 16: 0.97 / 0.99 against 0.93 / 0.94 for
+    //   one copy per row; D = 256: 0.96-0.98 against 0.94; D = 128, N = 8 / 16: 0.95 against
+    //   0.89 / 0.91; D = 64: 0.84-0.91 against 0.83.  Shapes it does not suit keep the kernels
+    //   above.
     PackGeom g;
+    if (!pack_geometry<dcp::kPackStages, dcp::kPackMaxTileRows>(a, dcp::kPackMinStageWords, g))
+        return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
+    const bool is_short = g.tiles <= 24 * g.cap;
+    if (!is_short && !(a.data_w >= 256 && (world_size == 3 || world_size == 4))) {
+        CUtensorMap map;
+        int dims = 0;
+        dcp::PackArgs t = a;
+        if (pack_tma_plan(t, cp_attn_out, H, D, es, out_stride_b, out_stride_h, map, dims))
+            return dims == 3 ? launch_pack_tma<3>(fn, t, map, stream) : launch_pack_tma<4>(fn, t, map, stream);
+    }
     if (a.data_w <= 32) {
         if (!pack_geometry<2, 256>(a, 12288, g)) return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
         return launch_pack<2, 256>(fn, a, g, true, stream);
     }
-    if (!pack_geometry<dcp::kPackStages, dcp::kPackMaxTileRows>(a, dcp::kPackMinStageWords, g))
-        return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
-    if (g.tiles <= 24 * g.cap) return launch_pack<dcp::kPackStages, dcp::kPackMaxTileRows>(fn, a, g, true, stream);
+    if (is_short) return launch_pack<dcp::kPackStages, dcp::kPackMaxTileRows>(fn, a, g, true, stream);
     if (a.data_w >= 256 && world_size <= 4) {
         PackGeom r;
         if (!pack_geometry<2, 256, true>(a, 12288, r)) return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
@@ -531,6 +661,8 @@ int32_t dcp_testing_split_shape(int32_t kind, int32_t N, int32_t chunks, int32_t
     out[3] = s.prefetch ? 1 : 0;
     return ok();
 }
+
+int32_t dcp_testing_last_pack_kernel(void) { return t_last_pack_kernel; }
 
 int32_t dcp_testing_pack_stalled(const void *cp_attn_out, const float *cp_attn_lse, void *send_buf, int64_t B,
                                  int64_t H, int64_t D, int32_t world_size, int32_t dtype, int64_t out_stride_b,

@@ -24,6 +24,7 @@
 // aligned.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (a type only; the library does not link the driver)
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -1184,6 +1185,12 @@ struct PackArgs {
     uint64_t wait_limit_ns;   // limit of each wait for a tile's copies (kWaitLimitNs)
     uint32_t stall_bytes;     // added to the byte count a CTA's first tile waits for: 0, except
                               // in the check of the timeout path (its wait then runs out)
+    // pack_tma_kernel only: tokens per box of the tensor map; tiles per rank; and, in the launch
+    // of each rank's last B mod tile_tokens tokens (one tile per rank), their first token and count
+    int32_t tile_tokens;
+    int32_t store_tokens;
+    int64_t tiles_per_rank;
+    int64_t first_token;
 };
 
 // Stores one landed tile: packed rows [i0, i0 + nrows) form the send range of words
@@ -1401,6 +1408,119 @@ __global__ void __launch_bounds__(THREADS) pack_kernel(const PackArgs a) {
         pack_store_tile(s_stage + (int)(k % kPackStages) * stage_w, a.dst, i0 * pitch, tile_rows_of(k), data_w, pitch,
                         lse_base, pitch_magic, tid, kPackThreads);
         __syncthreads();  // stage k % kPackStages is free for tile k + kPackStages
+    }
+    cp_async_wait<0>();
+}
+
+// The pack with each tile loaded by one tensor copy.  A tile is tile_tokens consecutive tokens
+// b0 .. of one rank, all Hr of its heads: a box [tile_tokens][Hr][D] of cp_attn_out, which the
+// tensor map `tmap` describes (3 dimensions {D, H, B}, or 4 {D/m, m, H, B} when a row is split
+// into m pieces of at most 256 elements), and packed rows [(rank B + b0) Hr, ...), one
+// contiguous range of the send buffer.  The box lands as rows back to back, as pack_store_tile
+// expects; the LSE words follow with 4-byte cp.async copies.  The whole-tile launch (TAIL =
+// false) covers tokens [0, B - B mod tile_tokens) of every rank, tile_tokens tokens a tile.  A
+// second launch (TAIL = true), one tile per rank, covers the tokens left: its tiles start at
+// first_token and store store_tokens tokens, and the box reaches past token B - 1, which the copy
+// fills with zeros and still counts.  Waits, the abort path and the stall hook are those of
+// pack_kernel.  STAGES tiles in flight per CTA; tiles of about 64 KiB with 2 stages measured best
+// (one CTA per SM).
+template <int STAGES, int THREADS, int DIMS, bool TAIL>
+__global__ void __launch_bounds__(THREADS) pack_tma_kernel(const __grid_constant__ CUtensorMap tmap, const PackArgs a) {
+    extern __shared__ __align__(128) uint4 s_tma_stage_v4[];
+    // the launch adds 128 bytes, so the stages can start on a 128-byte boundary
+    uint32_t *s_stage = reinterpret_cast<uint32_t *>(s_tma_stage_v4) + ((128u - (smem_addr(s_tma_stage_v4) & 127u)) & 127u) / 4;
+    __shared__ uint64_t s_full[STAGES];
+    __shared__ int s_abort;
+    const int tid = threadIdx.x;
+    const int Hr = (int)a.Hr;
+    const int ranks = (int)(a.rows / (a.B * a.Hr));
+    const int64_t tiles = (int64_t)ranks * a.tiles_per_rank;
+    const int64_t my_tiles = tiles > blockIdx.x ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int k = a.tile_tokens;
+    const int box_rows = k * Hr;
+    const int nrows = TAIL ? a.store_tokens * Hr : box_rows;  // rows each tile stores
+    const int data_w = a.data_w, pitch = a.row_pitch_w, stage_w = a.stage_w;
+    const int lse_base = box_rows * data_w;  // LSE words follow the box in a stage
+    const uint32_t box_bytes = (uint32_t)box_rows * (uint32_t)data_w * 4u;
+    const uint64_t tmap_addr = reinterpret_cast<uint64_t>(&tmap);
+
+    // (an offset added to b0 in the whole-tile launch cost about 7% at 1 KiB rows, measured)
+    auto tile_of = [&](int64_t kk, int &rank, int64_t &b0) {
+        const int64_t t = blockIdx.x + kk * gridDim.x;
+        rank = (int)(t / a.tiles_per_rank);
+        if constexpr (TAIL)
+            b0 = a.first_token;  // one tile per rank
+        else
+            b0 = (t - (int64_t)rank * a.tiles_per_rank) * k;
+    };
+    auto issue = [&](int64_t kk) {
+        int rank;
+        int64_t b0;
+        tile_of(kk, rank, b0);
+        const int slot = (int)(kk % STAGES);
+        uint32_t *stage = s_stage + slot * stage_w;
+        if (tid == 0) {
+            fence_proxy_async();
+            mbar_arrive_expect_tx(&s_full[slot], box_bytes + (kk == 0 ? a.stall_bytes : 0u));
+            if constexpr (DIMS == 3) {
+                asm volatile(
+                    "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+                    "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(stage)),
+                    "l"(tmap_addr), "r"(0), "r"(rank * Hr), "r"((int)b0), "r"(smem_addr(&s_full[slot]))
+                    : "memory");
+            } else {
+                asm volatile(
+                    "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+                    "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_addr(stage)),
+                    "l"(tmap_addr), "r"(0), "r"(0), "r"(rank * Hr), "r"((int)b0), "r"(smem_addr(&s_full[slot]))
+                    : "memory");
+            }
+        }
+        for (int r = tid; r < nrows; r += THREADS) {
+            const int64_t b = b0 + r / Hr;
+            cp_async_word(stage + lse_base + r, a.lse + b * a.lse_stride_b + rank * Hr + r % Hr);
+        }
+    };
+
+    if (tid == 0) {
+        for (int st = 0; st < STAGES; ++st) mbar_init(&s_full[st], 1);
+        mbar_fence_init();
+        s_abort = 0;
+    }
+    __syncthreads();
+    if (smem_addr(s_stage) & 127u) {  // a tensor copy needs a 128-byte aligned destination: none issued
+        if (tid == 0) atomicAdd(&g_wait_timeouts, 1ull);
+        return;
+    }
+#pragma unroll
+    for (int kk = 0; kk < STAGES - 1; ++kk) {
+        if (kk < my_tiles) issue(kk);
+        cp_async_commit();
+    }
+    for (int64_t kk = 0; kk < my_tiles; ++kk) {
+        if (kk + STAGES - 1 < my_tiles) issue(kk + STAGES - 1);
+        cp_async_commit();
+        cp_async_wait<STAGES - 1>();  // this thread's LSE copies of tile kk have landed
+        if (!mbar_wait_bounded(&s_full[(int)(kk % STAGES)], (uint32_t)((kk / STAGES) & 1), a.wait_limit_ns))
+            s_abort = 1;
+        __syncthreads();
+        if (s_abort) {
+            // as in pack_kernel: counted once, then wait (bounded) for every tile in flight
+            if (tid == 0) {
+                atomicAdd(&g_wait_timeouts, 1ull);
+                for (int64_t q = kk; q < kk + STAGES && q < my_tiles; ++q)
+                    mbar_wait_bounded(&s_full[(int)(q % STAGES)], (uint32_t)((q / STAGES) & 1), a.wait_limit_ns);
+            }
+            cp_async_wait<0>();
+            return;
+        }
+        int rank;
+        int64_t b0;
+        tile_of(kk, rank, b0);
+        const int64_t i0 = ((int64_t)rank * a.B + b0) * Hr;
+        pack_store_tile(s_stage + (int)(kk % STAGES) * stage_w, a.dst, i0 * pitch, nrows, data_w, pitch, lse_base,
+                        a.pitch_magic, tid, THREADS);
+        __syncthreads();  // stage kk % STAGES is free for tile kk + STAGES
     }
     cp_async_wait<0>();
 }

@@ -1,9 +1,9 @@
 /*
  * dcp_testing.h -- test hooks of libdcpcombine.so: one makes the timeout path of the pack
- * kernel's bounded wait run, so that a test can check it without faulting or hanging a
+ * kernels' bounded waits run, so that a test can check it without faulting or hanging a
  * GPU; one reports the launch shape the host picks for a split-layout combine, so that the
- * shape rules can be checked without a GPU.  Not part of the combine; no page has a
- * counterpart.
+ * shape rules can be checked without a GPU; one reports which pack kernel ran.  Not part of
+ * the combine; no page has a counterpart.
  */
 #ifndef DCP_TESTING_H
 #define DCP_TESTING_H
@@ -39,6 +39,16 @@ int32_t dcp_testing_pack_stalled(const void *cp_attn_out, const float *cp_attn_l
  * [1, DCP_MAX_SHARDS], chunks < 1 or a null `out`.
  */
 int32_t dcp_testing_split_shape(int32_t kind, int32_t N, int32_t chunks, int32_t *out);
+
+/*
+ * Which kernel the calling host thread's last dcp_pack (or dcp_testing_pack_stalled) launched,
+ * so that a test can check the path it covers: 0 = none yet (or an empty call), 1 = pack_kernel
+ * with one bulk copy per row, 2 = pack_kernel copying a token's contiguous heads as runs,
+ * 3 = pack_kernel with tiles in rank-fastest order, 4 = pack_tma_kernel with a 3-dimensional
+ * tensor map (rows of at most 256 elements), 5 = pack_tma_kernel with each row split into
+ * pieces (4 dimensions).  Needs no arguments and cannot fail.
+ */
+int32_t dcp_testing_last_pack_kernel(void);
 
 #ifdef __cplusplus
 }

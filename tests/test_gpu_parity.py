@@ -536,11 +536,11 @@ def test_pack_head_runs(o, B, H, D, ws, dtype):
     assert dcp.dcp_wait_timeouts() == 0
 
 
-@pytest.mark.parametrize("B,H,D,ws,dtype,pad", [(8000, 32, 512, 2, "bf16", 0), (4000, 64, 512, 4, "bf16", 0),
+@pytest.mark.parametrize("B,H,D,ws,dtype,pad", [(3000, 96, 512, 3, "bf16", 0), (4000, 64, 512, 4, "bf16", 0),
                                                (4000, 64, 256, 4, "fp32", 0), (2000, 128, 512, 4, "fp16", 0),
                                                (4000, 64, 512, 4, "bf16", 8)])
 def test_pack_rank_fast_order(o, B, H, D, ws, dtype, pad):
-    """Long launches of rows of 1 KiB and more for at most 4 ranks, where the pack's tiles run
+    """Long launches of rows of 1 KiB and more for 3 or 4 ranks, where the pack's tiles run
     in rank-fastest order and never straddle a rank (each rank's last tile is partial here):
     bit-exact against the oracle, with guard bands around the send buffer.  pad > 0: heads
     `D + pad` elements apart, so every row is a copy of its own."""
@@ -553,6 +553,7 @@ def test_pack_rank_fast_order(o, B, H, D, ws, dtype, pad):
     P = dcp.dcp_lse_pack_dim(dt)
     send = Guarded((ws, B, H // ws, D + P), dt)
     dcp.dcp_pack(big.cuda()[:, :, :D], lse.cuda(), send.tensor, ws)
+    assert dcp.library().dcp_testing_last_pack_kernel() == 3   # pack_kernel, rank-fastest tiles
     send.check()
     ref = o.pack(raw(out.contiguous()), raw(lse), ws, ORACLE_CODE[dt])
     assert np.array_equal(bits(send.tensor.cpu()), bits(ref))
