@@ -599,25 +599,30 @@ int32_t pack_impl(const char *fn, const void *cp_attn_out, const float *cp_attn_
     //   D = 512: 0.91 against 0.85; N = 2, B = 16384, D = 128: 0.88 against 0.80) and lose in
     //   longer ones, where one copy per row keeps more copies in flight (N = 16, B = 16384:
     //   D = 512 0.94 against 0.87, D = 128 0.91 against 0.85).
-    // * Longer launches of rows of 1 KiB and more for 3 or 4 ranks: 2 stages of up to 48 KiB,
-    //   tiles in rank-fastest order, so that the tiles in flight read all ranks of the same
-    //   tokens (D = 512, N = 4: 0.94 against 0.93 for the tensor copies below and 0.90 in rank
-    //   order; with 8 and 16 ranks this order lost, 0.89-0.91 against 0.92-0.96).
-    // * Longer launches otherwise: one tensor copy per tile of about 64 KiB (tokens x all heads of a
-    //   rank), 2 stages, one CTA per SM: D = 512, N = 8 / 16: 0.97 / 0.99 against 0.93 / 0.94 for
-    //   one copy per row; D = 256: 0.96-0.98 against 0.94; D = 128, N = 8 / 16: 0.95 against
-    //   0.89 / 0.91; D = 64: 0.84-0.91 against 0.83.  Shapes it does not suit keep the kernels
-    //   above.
+    // * Longer launches: one tensor copy per tile of about 64 KiB (tokens x all heads of a rank),
+    //   2 stages, one CTA per SM: N = 16, B = 16384: D = 512 1.00 against 0.94 for one copy per
+    //   row, D = 128 0.94 against 0.91; N = 8, B = 16384: D = 512 0.98, D = 256 0.97, D = 128
+    //   0.96 against 0.89; N = 3 / 4, B = 16384, D = 512: 0.98 / 0.94 against 0.92 / 0.91 for
+    //   the rank-fast order below; D = 64: 0.84-0.91 against 0.83.
+    // * Except rows of 1 KiB and more for 3 or 4 ranks in under ~64 tensor tiles per SM: 2 stages
+    //   of up to 48 KiB, tiles in rank-fastest order, so that the tiles in flight read all ranks
+    //   of the same tokens (N = 4, B = 4096, D = 512: 0.93 against 0.89 for the tensor copies).
+    //   Shapes the tensor copy does not suit also take the kernels above or this one.
     PackGeom g;
     if (!pack_geometry<dcp::kPackStages, dcp::kPackMaxTileRows>(a, dcp::kPackMinStageWords, g))
         return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
     const bool is_short = g.tiles <= 24 * g.cap;
-    if (!is_short && !(a.data_w >= 256 && (world_size == 3 || world_size == 4))) {
+    if (!is_short) {
         CUtensorMap map;
         int dims = 0;
         dcp::PackArgs t = a;
-        if (pack_tma_plan(t, cp_attn_out, H, D, es, out_stride_b, out_stride_h, map, dims))
-            return dims == 3 ? launch_pack_tma<3>(fn, t, map, stream) : launch_pack_tma<4>(fn, t, map, stream);
+        if (pack_tma_plan(t, cp_attn_out, H, D, es, out_stride_b, out_stride_h, map, dims)) {
+            const int64_t tma_tiles = (int64_t)world_size * ((a.B + t.tile_tokens - 1) / t.tile_tokens);
+            const bool rank_fast = a.data_w >= 256 && (world_size == 3 || world_size == 4) &&
+                                   tma_tiles < 64 * (int64_t)sm_count();
+            if (!rank_fast)
+                return dims == 3 ? launch_pack_tma<3>(fn, t, map, stream) : launch_pack_tma<4>(fn, t, map, stream);
+        }
     }
     if (a.data_w <= 32) {
         if (!pack_geometry<2, 256>(a, 12288, g)) return fail(DCP_ERR_CUDA, "%s: cannot reserve shared memory", fn);
