@@ -114,3 +114,34 @@ def test_tensor_pack_stalled_wait_is_counted_and_the_device_stays_usable(o):
     assert dcp.dcp_wait_timeouts() == 0
     ref = o.pack(raw(out), raw(lse), ws, orc.BF16)
     assert np.array_equal(bits(send2.cpu()), bits(ref))
+
+
+def test_tensor_pack_in_a_cuda_graph(o):
+    """Both launches of a tensor-copy pack (whole tiles and the per-rank tail), captured once in
+    a CUDA graph with their tensor map and replayed on new contents of the same buffers."""
+    B, H, D, ws = 2001, 128, 512, 8
+    cp_out = torch.empty((B, H, D), dtype=torch.bfloat16, device="cuda")
+    cp_lse = torch.empty((B, H), device="cuda")
+    send = torch.empty((ws, B, H // ws, D + 2), dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):  # per-device set-up before capture
+            dcp.dcp_pack(cp_out, cp_lse, send, ws)
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        dcp.dcp_pack(cp_out, cp_lse, send, ws)
+    assert dcp.library().dcp_testing_last_pack_kernel() == TENSOR_4D
+    for seed in (41, 42):
+        gen = torch.Generator().manual_seed(seed)
+        h_out = torch.randn(B, H, D, generator=gen).to(torch.bfloat16)
+        h_lse = torch.randn(B, H, generator=gen)
+        cp_out.copy_(h_out)
+        cp_lse.copy_(h_lse)
+        send.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        ref = o.pack(raw(h_out), raw(h_lse), ws, orc.BF16)
+        assert np.array_equal(bits(send.cpu()), bits(ref))
+    assert dcp.dcp_wait_timeouts() == 0
