@@ -112,7 +112,14 @@ int32_t dcp_lse_pack_dim(int32_t dtype);
  * 16/elemsize and >= 1 (else DCP_ERR_MISALIGNED / DCP_ERR_INVALID_ARG);
  * cp_attn_lse 4-byte aligned, lse_stride_b >= H.
  *
- * The kernel waits for its bulk copies with a time limit; a wait that runs out
+ * Long calls load each tile (consecutive tokens x all heads of one rank, about
+ * 64 KiB) with one tensor copy, through a tensor map the call encodes with the
+ * driver's cuTensorMapEncodeTiled (found through cudaGetDriverEntryPoint; the
+ * library does not link the driver); such a call may launch two kernels, the
+ * second for each rank's last B mod (tokens per tile) tokens.  Other calls, and
+ * any whose map the driver refuses, copy rows with bulk copies.  Same result.
+ *
+ * The kernels wait for their copies with a time limit; a wait that runs out
  * (never, while the copies work) leaves this call's send_buf incomplete and
  * is counted by dcp_wait_timeouts, and the call still returns DCP_OK (it
  * returns before the kernel runs).  A caller that must be sure of send_buf
@@ -259,9 +266,11 @@ int32_t dcp_unpack_combine(const void *recv_buf, void *result, float *global_lse
 
 /*
  * Pack CTAs whose wait timed out on the current device since the last reset.  dcp_pack
- * waits for its bulk copies with a limit of one second per wait; when a wait runs out the
- * CTA is counted here and stops (after waiting, bounded, for the copies it has issued), so
- * the send buffer of that call is incomplete.  A nonzero count therefore means a result is
+ * waits for its bulk and tensor copies with a limit of one second per wait; when a wait runs
+ * out the CTA is counted here and stops (after waiting, bounded, for the copies it has
+ * issued), so the send buffer of that call is incomplete.  A tensor-copy CTA whose shared
+ * memory cannot be placed on a 128-byte boundary is counted too and copies nothing (the
+ * launch reserves the room to align it, so this does not happen).  A nonzero count therefore means a result is
  * invalid (it never happens when the copies work).  Synchronises the device (the counter is
  * read from device memory); with reset != 0 the counter is cleared afterwards.  Returns
  * DCP_ERR_CUDA if the read fails.

@@ -62,6 +62,8 @@ TENSOR_CASES = [  # B, H, D, world_size, dtype, kernel expected
     (2001, 128, 256, 8, "fp32", TENSOR_3D),   # 1 KiB fp32 rows of 256 elements, k = 4
     (3601, 4, 8192, 2, "fp32", TENSOR_4D),    # 32 KiB rows in 32 pieces, 2 heads: one token a tile
     (2001, 128, 512, 16, "bf16", TENSOR_4D),  # 8 heads per rank, k = 8
+    (8001, 128, 256, 64, "bf16", TENSOR_3D),  # 64 ranks of 2 heads, k = 64
+    (8001, 256, 64, 1, "bf16", TENSOR_3D),    # 256 heads per rank (the box's limit), k = 2
     (3001, 256, 512, 4, "bf16", TENSOR_4D),   # 4 ranks of 64 heads, k = 1: 12004 tiles, over 64 per SM
     (1001, 256, 512, 4, "bf16", RANK_FAST),   # ... 4004 tiles: 4 ranks of 1 KiB rows keep the rank-fast order
     (2001, 128, 512, 1, "bf16", RANK_FAST),   # one rank: 128 KiB per token, over a tile
