@@ -196,12 +196,14 @@ constexpr int kPackTmaBoxBytes = 65536;  // about 64 KiB of rows per tile
 constexpr int kPackTmaMaxStageW = ((kPackTmaBoxBytes / 4 + kPackTmaBoxBytes / 16 + 4) + 31) & ~31;
 
 // A tensor map and tile shape for pack_tma_kernel, or false when the shape does not suit it
-// (more than 256 heads per rank, a token's heads over 64 KiB, no row split into pieces of at
-// most 256 elements and a multiple of 16 bytes, or an encoding the driver refuses).
+// (more than 256 heads per rank, a token's heads over 64 KiB, B or H beyond a 32-bit
+// coordinate, no row split into pieces of at most 256 elements and a multiple of 16 bytes, or
+// an encoding the driver refuses).
 bool pack_tma_plan(dcp::PackArgs &a, const void *cp_attn_out, int64_t H, int64_t D, int es, int64_t out_stride_b,
                    int64_t out_stride_h, CUtensorMap &map, int &dims) {
     const int64_t row_bytes = (int64_t)a.data_w * 4;
     if (a.Hr > 256 || a.Hr * row_bytes > kPackTmaBoxBytes) return false;
+    if (a.B > INT32_MAX || H > INT32_MAX) return false;  // tensor-copy coordinates are 32-bit
     int64_t k = kPackTmaBoxBytes / (a.Hr * row_bytes);
     if (k > 256) k = 256;
     if (k > a.B) k = a.B;
