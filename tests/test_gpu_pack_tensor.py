@@ -27,25 +27,29 @@ def o() -> orc.Oracle:
     return orc.load()
 
 
-def _pack_case(o, B, H, D, ws, dtype, pad_h=0, pad_b=0, seed=0):
+def _pack_case(o, B, H, D, ws, dtype, pad_h=0, pad_b=0, seed=0, lse_pad=0):
     """Packs a [B, H, D] view whose heads are D + pad_h elements apart and whose tokens are
-    H * (D + pad_h) + pad_b apart; returns the kernel that ran after checking the bits."""
+    H * (D + pad_h) + pad_b apart, with LSE rows H + lse_pad apart; returns the kernel that ran
+    after checking the bits."""
     dt = torch_dtype(dtype)
     gen = torch.Generator().manual_seed(seed or B * 3 + H * 5 + D * 7 + ws)
     per_b = H * (D + pad_h) + pad_b
     flat = torch.randn(B * per_b, generator=gen).to(dt)
     view = flat.as_strided((B, H, D), (per_b, D + pad_h, 1))
-    lse = torch.randn(B, H, generator=gen)
+    lse_big = torch.randn(B, H + lse_pad, generator=gen)
+    lse = lse_big[:, :H]
     lse.view(torch.int32)[0, 0] = 0x7FC0ABCD            # NaN payload must survive
     lse[B - 1, H - 1] = float("-inf")
     d_flat = flat.cuda()
     d_view = d_flat.as_strided((B, H, D), (per_b, D + pad_h, 1))
+    d_lse = lse_big.cuda()[:, :H]
+    assert d_lse.stride() == (H + lse_pad, 1)
     P = dcp.dcp_lse_pack_dim(dt)
     send = Guarded((ws, B, H // ws, D + P), dt)
-    dcp.dcp_pack(d_view, lse.cuda(), send.tensor, ws)
+    dcp.dcp_pack(d_view, d_lse, send.tensor, ws)
     kernel = dcp.library().dcp_testing_last_pack_kernel()
     send.check()
-    ref = o.pack(raw(view.contiguous()), raw(lse), ws, ORACLE_CODE[dt])
+    ref = o.pack(raw(view.contiguous()), raw(lse.contiguous()), ws, ORACLE_CODE[dt])
     assert np.array_equal(bits(send.tensor.cpu()), bits(ref))
     assert dcp.dcp_wait_timeouts() == 0
     return kernel
@@ -76,14 +80,15 @@ def test_tensor_pack(o, B, H, D, ws, dtype, kernel):
     assert _pack_case(o, B, H, D, ws, dtype) == kernel
 
 
-@pytest.mark.parametrize("B,H,D,ws,dtype,pad_h,pad_b,kernel", [
-    (2001, 128, 512, 8, "bf16", 8, 0, TENSOR_4D),    # heads D + 8 apart
-    (8001, 128, 128, 16, "fp16", 0, 64, TENSOR_3D),  # tokens 64 elements more than H D apart
-    (2001, 128, 256, 8, "fp32", 4, 12, TENSOR_3D),   # both
+@pytest.mark.parametrize("B,H,D,ws,dtype,pad_h,pad_b,lse_pad,kernel", [
+    (2001, 128, 512, 8, "bf16", 8, 0, 0, TENSOR_4D),    # heads D + 8 apart
+    (8001, 128, 128, 16, "fp16", 0, 64, 0, TENSOR_3D),  # tokens 64 elements more than H D apart
+    (2001, 128, 256, 8, "fp32", 4, 12, 0, TENSOR_3D),   # both
+    (4001, 128, 256, 8, "bf16", 0, 0, 3, TENSOR_3D),    # LSE rows H + 3 apart
 ])
-def test_tensor_pack_strided(o, B, H, D, ws, dtype, pad_h, pad_b, kernel):
+def test_tensor_pack_strided(o, B, H, D, ws, dtype, pad_h, pad_b, lse_pad, kernel):
     """The tensor map takes the head and token strides, so strided inputs keep the kernel."""
-    assert _pack_case(o, B, H, D, ws, dtype, pad_h, pad_b) == kernel
+    assert _pack_case(o, B, H, D, ws, dtype, pad_h, pad_b, lse_pad=lse_pad) == kernel
 
 
 def test_tensor_pack_stalled_wait_is_counted_and_the_device_stays_usable(o):
