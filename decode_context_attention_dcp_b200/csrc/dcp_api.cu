@@ -199,17 +199,25 @@ constexpr int kPackTmaMaxStageW = ((kPackTmaBoxBytes / 4 + kPackTmaBoxBytes / 16
 // (more than 256 heads per rank, a token's heads over 64 KiB, B or H beyond a 32-bit
 // coordinate, no row split into pieces of at most 256 elements and a multiple of 16 bytes, or
 // an encoding the driver refuses).
+// The tile shape alone: k tokens per tile (at most 256, at most B, k Hr rows within 64 KiB) and
+// the row split into m pieces (the fewest of at most 256 elements each, D a multiple of m, a
+// piece a multiple of 16 bytes); false when no such shape exists.
+bool pack_tma_shape(int64_t Hr, int64_t D, int es, int64_t B, int64_t &k, int64_t &m) {
+    const int64_t row_bytes = D * es;
+    if (Hr < 1 || B < 1 || D < 1 || Hr > 256 || Hr * row_bytes > kPackTmaBoxBytes) return false;
+    k = kPackTmaBoxBytes / (Hr * row_bytes);
+    if (k > 256) k = 256;
+    if (k > B) k = B;
+    m = (D + 255) / 256;
+    while (m <= 256 && (D % m != 0 || ((D / m) * es) % 16 != 0)) ++m;
+    return m <= 256;
+}
+
 bool pack_tma_plan(dcp::PackArgs &a, const void *cp_attn_out, int64_t H, int64_t D, int es, int64_t out_stride_b,
                    int64_t out_stride_h, CUtensorMap &map, int &dims) {
-    const int64_t row_bytes = (int64_t)a.data_w * 4;
-    if (a.Hr > 256 || a.Hr * row_bytes > kPackTmaBoxBytes) return false;
     if (a.B > INT32_MAX || H > INT32_MAX) return false;  // tensor-copy coordinates are 32-bit
-    int64_t k = kPackTmaBoxBytes / (a.Hr * row_bytes);
-    if (k > 256) k = 256;
-    if (k > a.B) k = a.B;
-    int64_t m = (D + 255) / 256;  // pieces per row
-    while (m <= 256 && (D % m != 0 || ((D / m) * es) % 16 != 0)) ++m;
-    if (m > 256) return false;
+    int64_t k = 0, m = 0;
+    if (!pack_tma_shape(a.Hr, D, es, a.B, k, m)) return false;
     PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
     if (!encode) return false;
     const CUtensorMapDataType type = es == 4 ? CU_TENSOR_MAP_DATA_TYPE_UINT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
@@ -670,6 +678,21 @@ int32_t dcp_testing_split_shape(int32_t kind, int32_t N, int32_t chunks, int32_t
 }
 
 int32_t dcp_testing_last_pack_kernel(void) { return t_last_pack_kernel; }
+
+int32_t dcp_testing_pack_tensor_shape(int64_t Hr, int64_t D, int32_t dtype, int64_t B, int32_t *out) {
+    if (dtype < 0 || dtype > 2 || Hr < 1 || D < 1 || B < 1 || !out)
+        return fail(DCP_ERR_INVALID_ARG, "dcp_testing_pack_tensor_shape: Hr %lld, D %lld, dtype %d, B %lld",
+                    (long long)Hr, (long long)D, (int)dtype, (long long)B);
+    int64_t k = 0, m = 0;
+    if (pack_tma_shape(Hr, D, elem_size(dtype), B, k, m)) {
+        out[0] = (int32_t)k;
+        out[1] = (int32_t)m;
+        out[2] = m == 1 ? 3 : 4;
+    } else {
+        out[0] = out[1] = out[2] = 0;
+    }
+    return ok();
+}
 
 int32_t dcp_testing_pack_stalled(const void *cp_attn_out, const float *cp_attn_lse, void *send_buf, int64_t B,
                                  int64_t H, int64_t D, int32_t world_size, int32_t dtype, int64_t out_stride_b,

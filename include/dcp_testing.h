@@ -2,8 +2,8 @@
  * dcp_testing.h -- test hooks of libdcpcombine.so: one makes the timeout path of the pack
  * kernels' bounded waits run, so that a test can check it without faulting or hanging a
  * GPU; one reports the launch shape the host picks for a split-layout combine, so that the
- * shape rules can be checked without a GPU; one reports which pack kernel ran.  Not part of
- * the combine; no page has a counterpart.
+ * shape rules can be checked without a GPU; two report which pack kernel ran and the tensor
+ * pack's tile shape.  Not part of the combine; no page has a counterpart.
  */
 #ifndef DCP_TESTING_H
 #define DCP_TESTING_H
@@ -49,6 +49,18 @@ int32_t dcp_testing_split_shape(int32_t kind, int32_t N, int32_t chunks, int32_t
  * pieces (4 dimensions).  Needs no arguments and cannot fail.
  */
 int32_t dcp_testing_last_pack_kernel(void);
+
+/*
+ * The tile shape dcp_pack's tensor copies would take for Hr heads per rank of D elements of
+ * `dtype` and B tokens, without encoding a map (needs no GPU): out[0] = k, the tokens per tile
+ * (at most 256 and at most B, k x Hr rows within 64 KiB, the largest such k); out[1] = m, the
+ * pieces each row is split into (the fewest with D a multiple of m, at most 256 elements and a
+ * multiple of 16 bytes each); out[2] = the tensor map's dimensions (3 when m = 1, else 4).
+ * All three are 0 when no tile suits the shape (more than 256 heads, or one token's heads over
+ * 64 KiB).  Which launches use the shape also depends on the device (see dcp_pack).  Returns
+ * DCP_OK, or DCP_ERR_INVALID_ARG for a dtype outside 0..2, Hr, D or B < 1, or a null `out`.
+ */
+int32_t dcp_testing_pack_tensor_shape(int64_t Hr, int64_t D, int32_t dtype, int64_t B, int32_t *out);
 
 #ifdef __cplusplus
 }

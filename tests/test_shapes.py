@@ -106,3 +106,60 @@ def test_weight_sums_match_the_plain_combine(shapes):
             for kind in (VARLEN, PACK):
                 G = shapes[kind, N, c][0]
                 assert G == Gp or N <= 2 * min(G, Gp), (kind, N, c, G, Gp)
+
+
+# ---- the tensor-copy pack's tile shape (dcp_testing_pack_tensor_shape) ----------------------
+
+BOX_BYTES = 65536
+
+
+@pytest.fixture(scope="module")
+def tensor_shape():
+    fn = dcp.library().dcp_testing_pack_tensor_shape
+    fn.restype = ctypes.c_int32
+    fn.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int64, ctypes.POINTER(ctypes.c_int32)]
+    out = (ctypes.c_int32 * 3)()
+
+    def shape(Hr, D, dtype, B):
+        assert fn(Hr, D, dtype, B, out) == 0
+        return tuple(out)
+    return shape
+
+
+def test_tensor_shape_invalid_arguments():
+    fn = dcp.library().dcp_testing_pack_tensor_shape
+    out = (ctypes.c_int32 * 3)()
+    for args in [(0, 128, 0, 16), (4, 0, 0, 16), (4, 128, 3, 16), (4, 128, -1, 16), (4, 128, 0, 0)]:
+        assert fn(*args, out) == 1
+    assert fn(4, 128, 0, 16, None) == 1
+
+
+@pytest.mark.parametrize("dtype,es", [(0, 2), (1, 2), (2, 4)])
+def test_tensor_shape_rules(tensor_shape, dtype, es):
+    """For every row length the API accepts (D * elemsize a multiple of 16, up to 8192) and a
+    spread of head and token counts: the tile is the largest k <= min(256, B) whose k x Hr rows
+    fit 64 KiB, and each row is split into the fewest m pieces of at most 256 elements and a
+    multiple of 16 bytes; no tile at all past 256 heads or one token's heads over 64 KiB."""
+    step = 16 // es
+    for D in range(step, 8193, step):
+        # the expected split, by brute force over every divisor
+        m_ref = next((m for m in range(1, 257) if D % m == 0 and D // m <= 256 and (D // m * es) % 16 == 0), None)
+        for Hr in (1, 2, 3, 4, 7, 16, 64, 128, 255, 256, 257):
+            for B in (1, 3, 1000, 100000):
+                k, m, dims = tensor_shape(Hr, D, dtype, B)
+                if Hr > 256 or Hr * D * es > BOX_BYTES or m_ref is None:
+                    assert (k, m, dims) == (0, 0, 0), (D, Hr, B)
+                    continue
+                assert 1 <= k <= min(256, B) and k * Hr * D * es <= BOX_BYTES, (D, Hr, B, k)
+                assert k == min(256, B) or (k + 1) * Hr * D * es > BOX_BYTES, (D, Hr, B, k)
+                assert m == m_ref and dims == (3 if m == 1 else 4), (D, m, m_ref)
+
+
+def test_tensor_shape_examples(tensor_shape):
+    """The shapes the bench and sweep workloads take (16 heads per rank, bf16)."""
+    assert tensor_shape(16, 512, 0, 16384) == (4, 2, 4)     # 4 tokens x 16 heads x 2 pieces of 256
+    assert tensor_shape(16, 128, 0, 16384) == (16, 1, 3)
+    assert tensor_shape(16, 64, 0, 32768) == (32, 1, 3)
+    assert tensor_shape(2, 8192, 2, 3601) == (1, 32, 4)     # fp32: 32 KiB rows in 32 pieces
+    assert tensor_shape(64, 512, 0, 3001) == (1, 2, 4)      # exactly 64 KiB per token
+    assert tensor_shape(128, 512, 0, 2001) == (0, 0, 0)     # 128 KiB per token: no tile
