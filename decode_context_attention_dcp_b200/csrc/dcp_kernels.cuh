@@ -12,6 +12,8 @@
 //                                      data (packed rows of at most 1 KiB)
 //   group_pack_kernel                  split merge written as 4-row spans of packed send rows
 //   pack_kernel                        output rows + fp32 LSE -> packed rows (bulk copies)
+//   pack_tma_kernel                    the same for long launches, each tile of tokens x a
+//                                      rank's heads loaded by one tensor copy
 //
 // The combine follows vLLM API docs, vllm.v1.attention.ops.dcp_alltoall,
 // _lse_weighted_combine; the packed layout [N, B, H/N, D + P] follows the same
